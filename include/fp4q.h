@@ -1,0 +1,187 @@
+/*
+ * fp4q.h -- C ABI of libfp4q.so: block-wise microscaling FP4 quantization of
+ * bf16 tensors on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three pages:
+ *  "Diagnosing FP4 inference: a layer-wise and block-wise sensitivity
+ *   analysis of NVFP4 and MXFP4", technical summary, Methodology (MXFP4: blocks
+ *   of 32 E2M1 values sharing an 8-bit exponent; NVFP4: blocks of 16 with a
+ *   scale and "max" calibration; weights kept in 16 bits, quantized on the fly
+ *   and dequantized for the compute);
+ *  "Bridging the Gap Between Promise and Performance for Microscaling FP4
+ *   Quantization", technical summary s1-s3 (E8M0 power-of-two scales, E4M3
+ *   scales, round-to-nearest, block-wise Hadamard rotations fused with the
+ *   quantization and the scale computation);
+ *  "Finer is better? Limits of micro-scaling formats in LLMs", Theoretical
+ *   framework, Contributions and Results (UE4M3 scales, smallest non-zero
+ *   2^-9; UE4M3 under a per-tensor scale; UE5M3; per-block and per-tensor MSE
+ *   split into non-max elements, block max and zero-rounded blocks).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are row-major and contiguous, [rows][cols].  A quantization block
+ *    is `block` consecutive elements of one row; a rotation acts on `rot`
+ *    consecutive elements of one row.  cols % block == 0 and, if rot > 0,
+ *    cols % rot == 0.  rows == 0 or cols == 0 is a valid empty tensor.
+ *  - Codes: 4-bit E2M1 nibbles (bit 3 = sign, bits 0-2 = magnitude index of
+ *    {0, 0.5, 1, 1.5, 2, 3, 4, 6}); byte j of the code buffer holds element 2j
+ *    in its low nibble and element 2j+1 in its high nibble: rows*cols/2 bytes.
+ *  - Scales: one byte per block, row-major [rows][cols/block].  E8M0: the
+ *    scale is 2^(byte-127).  UE4M3: unsigned E4M3 (bias 7, 0x7F NaN, max 448,
+ *    min 2^-9), block scale S = fp32(decode(byte) * G).  UE5M3: unsigned E5M3
+ *    (bias 15, 0xFF NaN, max 114688, min 2^-17), S = fp32(decode(byte) * G).
+ *  - G is the FP32 per-tensor scale (1 when none is used).
+ *  - All pointers except `stream` are DEVICE pointers owned by the caller; the
+ *    library allocates no memory.  `stream` is a cudaStream_t passed as void*
+ *    (NULL = the legacy default stream).  Every call only enqueues work on
+ *    that stream and returns; outputs are valid once the stream reaches it.
+ *  - Alignment: bf16 tensors and code buffers 32 bytes; scale and per-block
+ *    MSE buffers 16 bytes; gscale 4 bytes; terms and workspace 8 bytes.
+ *  - Errors: invalid arguments return a negative fp4q_status before anything
+ *    is enqueued.  A failed launch returns FP4Q_ERR_CUDA.  No call ever
+ *    synchronizes the device.  Inputs must be finite: a block holding NaN or
+ *    Inf gets an unspecified scale byte and codes (no fault).
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP4Q_API __attribute__((visibility("default")))
+#else
+#define FP4Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4Q_OK = 0,
+    FP4Q_ERR_NULL = -1,        /* a required pointer is NULL                    */
+    FP4Q_ERR_SHAPE = -2,       /* negative size, or cols not a multiple of block/rot */
+    FP4Q_ERR_ALIGN = -3,       /* a pointer breaks the alignment rules above    */
+    FP4Q_ERR_UNSUPPORTED = -4, /* format / block / rot / mode combination        */
+    FP4Q_ERR_CUDA = -5,        /* a CUDA launch or runtime call failed           */
+    FP4Q_ERR_WORKSPACE = -6    /* workspace smaller than fp4q_block_mse_workspace_size */
+} fp4q_status;
+
+typedef enum {
+    FP4Q_SCALE_E8M0 = 0,       /* MXFP4 power-of-two scale                      */
+    FP4Q_SCALE_UE4M3 = 1,      /* NVFP4 unsigned E4M3 scale                     */
+    FP4Q_SCALE_UE5M3 = 2       /* unsigned E5M3 scale (min 2^-17)               */
+} fp4q_scale_fmt;
+
+typedef enum {
+    FP4Q_GLOBAL_NONE = 0,      /* G = 1 (always for E8M0; plain UE4M3 / UE5M3)  */
+    FP4Q_GLOBAL_COMPUTE = 1,   /* G = amax(|y|)/(6*448) (1 if amax = 0), written to *gscale */
+    FP4Q_GLOBAL_GIVEN = 2      /* G read from *gscale (must be finite and > 0)  */
+} fp4q_global_mode;
+
+typedef enum {
+    FP4Q_OUT_BF16 = 0,         /* dequantized values rounded to bf16 (RNE)      */
+    FP4Q_OUT_F32 = 1           /* dequantized values as fp32                    */
+} fp4q_out_dtype;
+
+/*
+ * fp4q_quantize -- rotate (optional), scale and round a bf16 tensor to FP4.
+ * ("Bridging the Gap", s3.4: rotation fused with quantization and scale
+ * computation; "Diagnosing FP4 inference", Methodology: "max" calibration.)
+ *
+ *  x       bf16 [rows][cols] input (device).
+ *  fmt     fp4q_scale_fmt.  block: power of two in [8, 256].
+ *  rot     0 (none) or 16, 32, 128: y = H_rot x / sqrt(rot) per run of rot
+ *          elements (Sylvester Hadamard), computed in fp32.
+ *  gmode   fp4q_global_mode; must be FP4Q_GLOBAL_NONE for E8M0.
+ *  codes   out: rows*cols/2 bytes.  scales: out, rows*cols/block bytes.
+ *  gscale  1 float: written in COMPUTE mode, read in GIVEN mode, ignored (may
+ *          be NULL) in NONE mode.
+ * Per block: m = max |y|; E8M0 S = 2^(floor(log2 m)-2); UE4M3/UE5M3
+ * s = nearest code to fp32(m / fp32(6 G)) (ties to even, saturating), S =
+ * fp32(decode(s) G).  Each nibble is the E2M1 value nearest to fp32(y / S)
+ * (correctly rounded quotient; ties to the even code; saturation at 6; sign
+ * kept); a block with S = 0 stores 0x0 nibbles.
+ */
+FP4Q_API int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                  int gmode, uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
+
+/*
+ * fp4q_tensor_amax -- amax = max |y| over the whole (optionally rotated)
+ * tensor, written as one float.  This is the first half of the per-tensor
+ * scale of COMPUTE mode ("Finer is better?", Results: UE4M3 with a dynamic
+ * per-tensor scale needs this extra pass).
+ */
+FP4Q_API int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax,
+                     void* stream);
+
+/*
+ * fp4q_global_scale -- *gscale = amax / (6 * 448) (correctly rounded fp32), or
+ * 1 when amax = 0: the per-tensor scale of COMPUTE mode from an absolute
+ * maximum that is already known (for instance one reduced across several
+ * shards of a tensor).  amax and gscale may be the same address.
+ * ("Finer is better?", Results: UE4M3 under a per-tensor scale.)
+ */
+FP4Q_API int fp4q_global_scale(const float* amax, float* gscale, void* stream);
+
+/*
+ * fp4q_dequantize -- v = fp32(decode(nibble) * S) ("Diagnosing FP4
+ * inference", Methodology: dequantized for the compute).
+ *  gscale   NULL means G = 1; otherwise G = *gscale (ignored for E8M0).
+ *  rot      0: v in the quantized (rotated) domain; 16/32/128: v is rotated
+ *           back, H_rot v / sqrt(rot) (the rotation is its own inverse).
+ *  out_dtype  FP4Q_OUT_BF16 (RNE of the fp32 value) or FP4Q_OUT_F32.
+ *  y        out: rows*cols values.
+ */
+FP4Q_API int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                    int64_t rows, int64_t cols, int fmt, int block, int rot, int out_dtype,
+                    void* y, void* stream);
+
+/*
+ * fp4q_block_mse -- quantization MSE per block and per tensor with the
+ * three-term split of "Finer is better?", Theoretical framework.
+ * Recomputes y from x (rotating when rot > 0) and v from codes/scales, then
+ *  block_mse[i] = sum_{j in block i} (y_j - v_j)^2 / block   (fp32; may be NULL)
+ *  terms[0..3]  = {total, non-max elements, block max, zero-rounded blocks},
+ *                 each a sum of squared errors over the tensor divided by
+ *                 rows*cols (fp64, device).  A block is zero-rounded when all
+ *                 of its dequantized values are 0; the block max is an element
+ *                 of largest |y|.
+ *  workspace    device scratch of at least fp4q_block_mse_workspace_size()
+ *               bytes, 8-byte aligned; its contents on entry do not matter.
+ * The per-tensor sums use a fixed reduction order (deterministic run to run).
+ */
+FP4Q_API int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,
+                   const float* gscale, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                   float* block_mse, double* terms, void* workspace, size_t ws_bytes,
+                   void* stream);
+
+/* Bytes of device workspace fp4q_block_mse needs for this shape (host only). */
+FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block);
+
+/*
+ * Element and scale codecs on their own, one value at a time ("Bridging the
+ * Gap", s1; "Finer is better?", Theoretical framework and Contributions).
+ * fp4q_e2m1_encode_f32: nibble of the E2M1 value nearest to r[i] (the rule of
+ *   fp4q_quantize with S = 1: ties to the even code, saturation at 6, sign
+ *   kept), packed like the code buffer (low nibble = even element).
+ * fp4q_scale_encode_f32: one scale byte per value.  UE4M3 / UE5M3: the code
+ *   nearest to s[i] >= 0 (ties to even, saturating at the largest finite
+ *   value).  E8M0: the byte fp4q_quantize stores for a block whose absolute
+ *   maximum is s[i] (2^(floor(log2 s) - 2), clamped to 2^-127).
+ * Inputs 4-byte aligned; outputs 4-byte aligned.
+ */
+FP4Q_API int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* stream);
+FP4Q_API int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, void* stream);
+
+/* Static text for a status code; never NULL. */
+FP4Q_API const char* fp4q_status_string(int status);
+
+/* ABI version of this header (incremented on any signature change). */
+FP4Q_API int fp4q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

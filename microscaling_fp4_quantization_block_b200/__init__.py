@@ -1,0 +1,223 @@
+"""Python binding of libfp4q.so (B200 block-wise microscaling FP4 quantization).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch supplies device memory and streams; each function below has
+the name of the C entry point it calls (see include/fp4q.h), takes CUDA
+tensors, allocates any output that is not given, checks the returned status
+and raises ``Fp4qError`` on failure.  There is no CPU fallback: if the
+library is missing, the first call raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp4q.so")
+
+# enums of include/fp4q.h
+FP4Q_OK = 0
+FP4Q_SCALE_E8M0, FP4Q_SCALE_UE4M3, FP4Q_SCALE_UE5M3 = 0, 1, 2
+FP4Q_GLOBAL_NONE, FP4Q_GLOBAL_COMPUTE, FP4Q_GLOBAL_GIVEN = 0, 1, 2
+FP4Q_OUT_BF16, FP4Q_OUT_F32 = 0, 1
+
+_FMT_NAMES = {"e8m0": FP4Q_SCALE_E8M0, "mxfp4": FP4Q_SCALE_E8M0, "ue4m3": FP4Q_SCALE_UE4M3,
+              "nvfp4": FP4Q_SCALE_UE4M3, "ue5m3": FP4Q_SCALE_UE5M3}
+_GMODE_NAMES = {"none": FP4Q_GLOBAL_NONE, "compute": FP4Q_GLOBAL_COMPUTE, "given": FP4Q_GLOBAL_GIVEN}
+
+
+class Fp4qError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fp4q_status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m microscaling_fp4_quantization_block_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "fp4q_quantize": (I, [P, I64, I64, I, I, I, I, P, P, P, P]),
+        "fp4q_tensor_amax": (I, [P, I64, I64, I, P, P]),
+        "fp4q_global_scale": (I, [P, P, P]),
+        "fp4q_dequantize": (I, [P, P, P, I64, I64, I, I, I, I, P, P]),
+        "fp4q_block_mse": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P, SZ, P]),
+        "fp4q_block_mse_workspace_size": (SZ, [I64, I64, I]),
+        "fp4q_e2m1_encode_f32": (I, [P, I64, P, P]),
+        "fp4q_scale_encode_f32": (I, [P, I64, I, P, P]),
+        "fp4q_status_string": (ctypes.c_char_p, [I]),
+        "fp4q_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raw pointer-level access); loaded on first use and
+    raising ImportError if libfp4q.so has not been built."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def _fmt(f) -> int:
+    return _FMT_NAMES[f.lower()] if isinstance(f, str) else int(f)
+
+
+def _gmode(g) -> int:
+    return _GMODE_NAMES[g.lower()] if isinstance(g, str) else int(g)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != FP4Q_OK:
+        raise Fp4qError(status, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("fp4q tensors must live on a CUDA device")
+
+
+def fp4q_version() -> int:
+    return lib().fp4q_version()
+
+
+def fp4q_status_string(status: int) -> str:
+    return lib().fp4q_status_string(status).decode()
+
+
+def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
+                  codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                  gscale: Optional[torch.Tensor] = None, stream=None
+                  ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """Quantize a 2-D bf16 CUDA tensor; returns (codes, scales, gscale)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    fmt, gmode = _fmt(fmt), _gmode(gmode)
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // block if block else 0), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode != FP4Q_GLOBAL_NONE:
+        gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    _need_cuda(codes, scales, gscale)
+    st = lib().fp4q_quantize(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(codes), _ptr(scales),
+                            _ptr(gscale), _stream(stream))
+    _check(st, "fp4q_quantize")
+    return codes, scales, gscale
+
+
+def fp4q_tensor_amax(x: torch.Tensor, rot: int = 0, amax: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    if amax is None:
+        amax = torch.empty((1,), dtype=torch.float32, device=x.device)
+    st = lib().fp4q_tensor_amax(_ptr(x), x.shape[0], x.shape[1], rot, _ptr(amax), _stream(stream))
+    _check(st, "fp4q_tensor_amax")
+    return amax
+
+
+def fp4q_global_scale(amax: torch.Tensor, gscale: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """G = amax / (6 * 448), or 1 if amax = 0 (device scalar in, device scalar out)."""
+    _need_cuda(amax)
+    if gscale is None:
+        gscale = torch.empty((1,), dtype=torch.float32, device=amax.device)
+    _check(lib().fp4q_global_scale(_ptr(amax), _ptr(gscale), _stream(stream)), "fp4q_global_scale")
+    return gscale
+
+
+def fp4q_dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[torch.Tensor],
+                    rows: int, cols: int, fmt, block: int, rot: int = 0,
+                    out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Dequantize codes/scales into a [rows, cols] bf16 or fp32 tensor."""
+    _need_cuda(codes, scales, gscale)
+    od = FP4Q_OUT_F32 if out_dtype == torch.float32 else FP4Q_OUT_BF16
+    if y is None:
+        y = torch.empty((rows, cols), dtype=torch.float32 if od == FP4Q_OUT_F32 else torch.bfloat16,
+                        device=codes.device)
+    st = lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(gscale), rows, cols, _fmt(fmt), block, rot,
+                              od, _ptr(y), _stream(stream))
+    _check(st, "fp4q_dequantize")
+    return y
+
+
+def fp4q_block_mse_workspace_size(rows: int, cols: int, block: int) -> int:
+    return int(lib().fp4q_block_mse_workspace_size(rows, cols, block))
+
+
+def fp4q_block_mse(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                   gscale: Optional[torch.Tensor], fmt, block: int, rot: int = 0,
+                   block_mse: Optional[torch.Tensor] = None, want_block_mse: bool = True,
+                   terms: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[Optional[torch.Tensor], torch.Tensor]:
+    """Per-block MSE (fp32) and terms [total, non-max, max, zero-rounded] (fp64)."""
+    _need_cuda(x, codes, scales, gscale)
+    x = x.contiguous()
+    rows, cols = x.shape
+    dev = x.device
+    if block_mse is None and want_block_mse:
+        block_mse = torch.empty((rows, cols // block), dtype=torch.float32, device=dev)
+    if terms is None:
+        terms = torch.empty((4,), dtype=torch.float64, device=dev)
+    ws = fp4q_block_mse_workspace_size(rows, cols, block)
+    if workspace is None:
+        workspace = torch.empty((ws,), dtype=torch.uint8, device=dev)
+    st = lib().fp4q_block_mse(_ptr(x), _ptr(codes), _ptr(scales), _ptr(gscale), rows, cols, _fmt(fmt),
+                             block, rot, _ptr(block_mse), _ptr(terms), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "fp4q_block_mse")
+    return block_mse, terms
+
+
+def fp4q_e2m1_encode_f32(r: torch.Tensor, packed: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    _need_cuda(r)
+    r = r.contiguous()
+    if packed is None:
+        packed = torch.empty((r.numel() // 2,), dtype=torch.uint8, device=r.device)
+    _check(lib().fp4q_e2m1_encode_f32(_ptr(r), r.numel(), _ptr(packed), _stream(stream)),
+           "fp4q_e2m1_encode_f32")
+    return packed
+
+
+def fp4q_scale_encode_f32(s: torch.Tensor, fmt, codes: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    _need_cuda(s)
+    s = s.contiguous()
+    if codes is None:
+        codes = torch.empty((s.numel(),), dtype=torch.uint8, device=s.device)
+    _check(lib().fp4q_scale_encode_f32(_ptr(s), s.numel(), _fmt(fmt), _ptr(codes), _stream(stream)),
+           "fp4q_scale_encode_f32")
+    return codes

@@ -1,0 +1,233 @@
+// fp4q_api.cu -- the C ABI of libfp4q.so: argument checks, then stream-ordered
+// launches.  Nothing here allocates device memory or synchronizes.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/fp4q.h"
+#include "fp4q_kernels.cuh"
+#include "fp4q_launch.h"
+
+namespace {
+
+using namespace fp4q;
+
+constexpr int kAbiVersion = 1;
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Shape / format checks common to every tensor entry point.  On success *n is
+// rows * cols.
+int check_shape(int64_t rows, int64_t cols, int fmt, int block, int rot, int64_t* n)
+{
+    if (rows < 0 || cols < 0) return FP4Q_ERR_SHAPE;
+    if (fmt != FP4Q_SCALE_E8M0 && fmt != FP4Q_SCALE_UE4M3 && fmt != FP4Q_SCALE_UE5M3)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!is_pow2(block) || block < 8 || block > 256) return FP4Q_ERR_UNSUPPORTED;
+    if (rot != 0 && rot != 16 && rot != 32 && rot != 128) return FP4Q_ERR_UNSUPPORTED;
+    if (cols % block != 0) return FP4Q_ERR_SHAPE;
+    if (rot != 0 && cols % rot != 0) return FP4Q_ERR_SHAPE;
+    if (cols != 0 && rows > INT64_MAX / 4 / cols) return FP4Q_ERR_SHAPE;
+    *n = rows * cols;
+    return FP4Q_OK;
+}
+
+// 1/sqrt(k) in fp64, split into an fp32 head and an fp32 tail.
+void rotation_constants(int rot, float* hi, float* lo)
+{
+    if (rot == 0) {
+        *hi = 1.0f;
+        *lo = 0.0f;
+        return;
+    }
+    const double c = 1.0 / std::sqrt((double)rot);
+    *hi = (float)c;
+    *lo = (float)(c - (double)*hi);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
+
+// amax(|y|) of the tensor into *dst (fp32 bits, via atomicMax on a zeroed slot).
+cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStream_t s)
+{
+    cudaError_t e = cudaMemsetAsync(dst, 0, sizeof(float), s);
+    if (e != cudaSuccess || n == 0) return e;
+    AmaxParams ap{};
+    ap.x = static_cast<const uint16_t*>(x);
+    ap.n = n;
+    ap.amax_bits = reinterpret_cast<unsigned int*>(dst);
+    rotation_constants(rot, &ap.c_hi, &ap.c_lo);
+    return launch_amax(rot, ap, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp4q_version(void) { return kAbiVersion; }
+
+const char* fp4q_status_string(int status)
+{
+    switch (status) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_NULL: return "a required pointer is NULL";
+    case FP4Q_ERR_SHAPE: return "bad shape: negative size, or cols not a multiple of block / rot";
+    case FP4Q_ERR_ALIGN: return "misaligned pointer (bf16 tensors and codes: 32 B; scales: 16 B)";
+    case FP4Q_ERR_UNSUPPORTED: return "unsupported format, block size, rotation or scale mode";
+    case FP4Q_ERR_CUDA: return "CUDA launch or runtime error";
+    case FP4Q_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+    }
+}
+
+int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                  uint8_t* codes, uint8_t* scales, float* gscale, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (gmode != FP4Q_GLOBAL_NONE && gmode != FP4Q_GLOBAL_COMPUTE && gmode != FP4Q_GLOBAL_GIVEN)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
+    if (gmode != FP4Q_GLOBAL_NONE) {
+        if (!gscale) return FP4Q_ERR_NULL;
+        if (!aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    }
+    if (n > 0) {
+        if (!x || !codes || !scales) return FP4Q_ERR_NULL;
+        if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)) return FP4Q_ERR_ALIGN;
+    }
+    cudaStream_t s = as_stream(stream);
+    if (gmode == FP4Q_GLOBAL_COMPUTE) {
+        cudaError_t e = enqueue_amax(x, n, rot, gscale, s);
+        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+        global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
+        if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    if (n == 0) return FP4Q_OK;
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.n = n;
+    p.codes = codes;
+    p.scales = scales;
+    p.gsrc = (gmode == FP4Q_GLOBAL_NONE) ? nullptr : gscale;
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
+    return cuda_status(launch_quantize(fmt, block, rot, p, s));
+}
+
+int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, FP4Q_SCALE_E8M0, 8, rot, &n);
+    if (st) return st;
+    if (!amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
+    if (!aligned(amax, 4) || (n > 0 && !aligned(x, 32))) return FP4Q_ERR_ALIGN;
+    return cuda_status(enqueue_amax(x, n, rot, amax, as_stream(stream)));
+}
+
+int fp4q_global_scale(const float* amax, float* gscale, void* stream)
+{
+    if (!amax || !gscale) return FP4Q_ERR_NULL;
+    if (!aligned(amax, 4) || !aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    global_scale_kernel<<<1, 1, 0, as_stream(stream)>>>(amax, gscale);
+    return cuda_status(cudaGetLastError());
+}
+
+int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t rows,
+                    int64_t cols, int fmt, int block, int rot, int out_dtype, void* y, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (out_dtype != FP4Q_OUT_BF16 && out_dtype != FP4Q_OUT_F32) return FP4Q_ERR_UNSUPPORTED;
+    if (gscale && !aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    if (n == 0) return FP4Q_OK;
+    if (!codes || !scales || !y) return FP4Q_ERR_NULL;
+    if (!aligned(codes, 32) || !aligned(scales, 16) || !aligned(y, 32)) return FP4Q_ERR_ALIGN;
+    DequantParams p{};
+    p.codes = codes;
+    p.scales = scales;
+    p.gsrc = gscale;
+    p.n = n;
+    p.fmt = fmt;
+    p.y = y;
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
+    return cuda_status(launch_dequantize(block, rot, out_dtype == FP4Q_OUT_F32, p, as_stream(stream)));
+}
+
+size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block)
+{
+    (void)block;
+    if (rows < 0 || cols < 0) return 0;
+    const int64_t n = rows * cols;
+    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    int64_t ctas = (tiles + kThreads / 32 - 1) / (kThreads / 32);
+    if (ctas < 1) ctas = 1;
+    if (ctas > kMaxMseCtas) ctas = kMaxMseCtas;
+    return (size_t)ctas * 4 * sizeof(double);
+}
+
+int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                   int64_t rows, int64_t cols, int fmt, int block, int rot, float* block_mse,
+                   double* terms, void* workspace, size_t ws_bytes, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (!terms || !workspace) return FP4Q_ERR_NULL;
+    if (n > 0 && (!x || !codes || !scales)) return FP4Q_ERR_NULL;
+    if (!aligned(terms, 8) || !aligned(workspace, 8)) return FP4Q_ERR_ALIGN;
+    if (gscale && !aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)))
+        return FP4Q_ERR_ALIGN;
+    if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
+    if (ws_bytes < fp4q_block_mse_workspace_size(rows, cols, block)) return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    double* partials = static_cast<double*>(workspace);
+    int grid = 0;
+    if (n > 0) {
+        grid = mse_grid(block, rot, n);
+        if (grid <= 0) return FP4Q_ERR_UNSUPPORTED;
+        MseParams p{};
+        p.x = static_cast<const uint16_t*>(x);
+        p.codes = codes;
+        p.scales = scales;
+        p.gsrc = gscale;
+        p.n = n;
+        p.fmt = fmt;
+        p.block_mse = block_mse;
+        p.partials = partials;
+        rotation_constants(rot, &p.c_hi, &p.c_lo);
+        if (launch_block_mse(block, rot, p, grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
+    return cuda_status(cudaGetLastError());
+}
+
+int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* stream)
+{
+    if (n < 0 || (n & 1)) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!r || !packed) return FP4Q_ERR_NULL;
+    if (!aligned(r, 4) || !aligned(packed, 4)) return FP4Q_ERR_ALIGN;
+    const int64_t work = (n + 7) / 8;
+    int grid = resident_grid((const void*)e2m1_encode_kernel, (work + kThreads - 1) / kThreads);
+    e2m1_encode_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(r, n, packed);
+    return cuda_status(cudaGetLastError());
+}
+
+int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, void* stream)
+{
+    if (n < 0) return FP4Q_ERR_SHAPE;
+    if (fmt != FP4Q_SCALE_E8M0 && fmt != FP4Q_SCALE_UE4M3 && fmt != FP4Q_SCALE_UE5M3)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (n == 0) return FP4Q_OK;
+    if (!s || !codes) return FP4Q_ERR_NULL;
+    if (!aligned(s, 4) || !aligned(codes, 4)) return FP4Q_ERR_ALIGN;
+    int grid = resident_grid((const void*)scale_encode_kernel, (n + kThreads - 1) / kThreads);
+    scale_encode_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(s, n, fmt, codes);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/fp4q.h declares, and rejects bad arguments on the host before it
+enqueues anything (these calls never reach the CUDA runtime)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4q.h")
+
+
+@pytest.fixture(scope="module")
+def fp4q():
+    from microscaling_fp4_quantization_block_b200 import build
+    build.build()
+    import microscaling_fp4_quantization_block_b200 as m
+    return m
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FP4Q_API\s+[\w\s\*]+?\b(fp4q_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ["fp4q_quantize", "fp4q_dequantize", "fp4q_block_mse", "fp4q_block_mse_workspace_size",
+                 "fp4q_tensor_amax", "fp4q_status_string", "fp4q_version"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(fp4q):
+    out = subprocess.run(["nm", "-D", "--defined-only", fp4q.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (fp4q_\w+)", out))
+    assert set(_declared()) <= exported
+    lib = ctypes.CDLL(fp4q.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(fp4q):
+    assert fp4q.fp4q_version() == 1
+    for st in range(0, -7, -1):
+        s = fp4q.fp4q_status_string(st)
+        assert s and s != "unknown status"
+    assert fp4q.fp4q_status_string(-99) == "unknown status"
+
+
+# Fake device addresses: never dereferenced, because every call below is
+# rejected by the host-side checks that run before any launch.
+A32 = 0x7F0000000000          # 32-byte aligned
+A4 = A32 + 4                  # 4-byte aligned only
+
+
+def test_quantize_rejects_bad_arguments(fp4q):
+    q = fp4q.lib().fp4q_quantize
+    E8, U4, U5 = 0, 1, 2
+    NONE, COMP, GIVEN = 0, 1, 2
+    assert q(A32, -1, 64, E8, 32, 0, NONE, A32, A32, None, None) == -2          # negative rows
+    assert q(A32, 4, 48, E8, 32, 0, NONE, A32, A32, None, None) == -2           # 48 % 32
+    assert q(A32, 4, 64, E8, 16, 128, NONE, A32, A32, None, None) == -2         # 64 % 128
+    assert q(A32, 4, 64, 3, 16, 0, NONE, A32, A32, None, None) == -4            # unknown format
+    assert q(A32, 4, 64, U4, 12, 0, NONE, A32, A32, None, None) == -4           # block not pow2
+    assert q(A32, 4, 512, U4, 512, 0, NONE, A32, A32, None, None) == -4         # block > 256
+    assert q(A32, 4, 512, U4, 4, 0, NONE, A32, A32, None, None) == -4           # block < 8
+    assert q(A32, 4, 64, U4, 16, 64, NONE, A32, A32, None, None) == -4          # rot 64 unsupported
+    assert q(A32, 4, 64, U4, 16, 0, 7, A32, A32, None, None) == -4              # unknown gmode
+    assert q(A32, 4, 64, E8, 32, 0, COMP, A32, A32, A32, None) == -4            # MX has no tensor scale
+    assert q(A32, 4, 64, U4, 16, 0, GIVEN, A32, A32, None, None) == -1          # gscale needed
+    assert q(None, 4, 64, U4, 16, 0, NONE, A32, A32, None, None) == -1
+    assert q(A32, 4, 64, U4, 16, 0, NONE, None, A32, None, None) == -1
+    assert q(A32, 4, 64, U4, 16, 0, NONE, A32, None, None, None) == -1
+    assert q(A32 + 16, 4, 64, U4, 16, 0, NONE, A32, A32, None, None) == -3      # x not 32-aligned
+    assert q(A32, 4, 64, U4, 16, 0, NONE, A32 + 8, A32, None, None) == -3
+    assert q(A32, 4, 64, U4, 16, 0, NONE, A32, A32 + 8, None, None) == -3       # scales not 16-aligned
+    assert q(A32, 4, 64, U4, 16, 0, GIVEN, A32, A32, A32 + 2, None) == -3
+    assert q(A32, 1 << 62, 1 << 8, U4, 16, 0, NONE, A32, A32, None, None) == -2  # overflow
+    # empty tensors are valid and enqueue nothing without a per-tensor scale
+    assert q(None, 0, 64, U4, 16, 0, NONE, None, None, None, None) == 0
+    assert q(None, 5, 0, E8, 32, 0, NONE, None, None, None, None) == 0
+    assert q(None, 0, 64, U5, 16, 32, GIVEN, None, None, A4, None) == 0
+
+
+def test_dequantize_and_mse_reject_bad_arguments(fp4q):
+    L = fp4q.lib()
+    assert L.fp4q_dequantize(A32, A32, None, 4, 64, 1, 16, 0, 2, A32, None) == -4       # bad out dtype
+    assert L.fp4q_dequantize(None, A32, None, 4, 64, 1, 16, 0, 0, A32, None) == -1
+    assert L.fp4q_dequantize(A32, A32, None, 4, 64, 1, 16, 0, 0, A32 + 16, None) == -3
+    assert L.fp4q_dequantize(None, None, None, 0, 64, 1, 16, 0, 0, None, None) == 0
+    ws = L.fp4q_block_mse_workspace_size(4, 64, 16)
+    assert ws >= 32 and ws % 8 == 0
+    assert L.fp4q_block_mse(A32, A32, A32, None, 4, 64, 1, 16, 0, None, A32, A32, ws - 8, None) == -6
+    assert L.fp4q_block_mse(A32, A32, A32, None, 4, 64, 1, 16, 0, None, None, A32, ws, None) == -1
+    assert L.fp4q_block_mse(A32, A32, A32, None, 4, 64, 1, 16, 0, A32 + 4, A32, A32, ws, None) == -3
+    assert L.fp4q_block_mse(A32, A32, A32, None, 4, 60, 1, 16, 0, None, A32, A32, ws, None) == -2
+    assert L.fp4q_tensor_amax(A32, 4, 64, 0, None, None) == -1
+    assert L.fp4q_tensor_amax(A32, 4, 64, 12, A32, None) == -4
+    assert L.fp4q_e2m1_encode_f32(A32, 7, A32, None) == -2                            # odd count
+    assert L.fp4q_scale_encode_f32(A32, 8, 9, A32, None) == -4
+    assert L.fp4q_e2m1_encode_f32(None, 0, None, None) == 0
+    assert L.fp4q_global_scale(None, A32, None) == -1
+    assert L.fp4q_global_scale(A32 + 2, A32, None) == -3
+
+
+def test_workspace_size_is_bounded(fp4q):
+    L = fp4q.lib()
+    small = L.fp4q_block_mse_workspace_size(1, 16, 16)
+    big = L.fp4q_block_mse_workspace_size(1 << 20, 1 << 14, 16)
+    assert small == 32
+    assert big == 4096 * 32
+    assert L.fp4q_block_mse_workspace_size(-1, 16, 16) == 0
+
+
+def test_binding_refuses_cpu_tensors(fp4q):
+    import torch
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fp4q.fp4q_quantize(x, "nvfp4", 16)
