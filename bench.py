@@ -3,8 +3,8 @@
 
 One step = the whole hot path over one batch of synthetic input: for every
 tensor of the workload, the per-tensor amax, the per-tensor scale, the fused
-(rotate+)scale+round+pack quantize kernel, dequantization and the per-block /
-per-tensor MSE with its three-term split.  Default workload: NVFP4 (block 16,
+(rotate+)scale+round+pack quantize kernel that also measures the per-block /
+per-tensor MSE with its three-term split, and dequantization.  Default workload: NVFP4 (block 16,
 UE4M3 block scales, FP32 per-tensor scale amax/(6*448)) on the nine Qwen2.5-7B
 MLP weights gate/up 18944x3584 and down 3584x18944 at sigma 0.005/0.02/0.05
 (611M elements, 1.22 GB of bf16 per step: larger than L2).
@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: max(3, steps // 20))")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-mse", action="store_true",
+                    help="measure the MSE with its own pass over x (fp4q_quantize + fp4q_block_mse)")
     return ap.parse_args(argv)
 
 
@@ -112,6 +114,7 @@ def bytes_per_element(block: int):
     return {
         "amax": 2.0,
         "quantize": 2.0 + 0.5 + 1.0 / block,
+        "quantize_mse": 2.0 + 0.5 + 1.0 / block + 4.0 / block,
         "dequantize": 0.5 + 1.0 / block + 2.0,
         "block_mse": 2.0 + 0.5 + 1.0 / block + 4.0 / block,
     }
@@ -126,10 +129,8 @@ class Pipeline:
     one kernel is the event before the next.
     """
 
-    STAGES_COMP = ("amax", "global_scale", "quantize", "dequantize", "block_mse")
-    STAGES_PLAIN = ("quantize", "dequantize", "block_mse")
 
-    def __init__(self, fq, items, device, stream):
+    def __init__(self, fq, items, device, stream, separate_mse=False):
         import torch
         self.fq, self.items, self.device = fq, items, device
         L = fq.lib()
@@ -156,17 +157,24 @@ class Pipeline:
             if comp:
                 seq.append(("amax", L.fp4q_tensor_amax, (x.data_ptr(), rows, cols, rot, p["amax"], sh)))
                 seq.append(("global_scale", L.fp4q_global_scale, (p["amax"], p["gscale"], sh)))
-            seq.append(("quantize", L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot,
-                                                      GIVEN if comp else NONE, p["codes"], p["scales"], g, sh)))
+            gm = GIVEN if comp else NONE
+            if separate_mse:
+                seq.append(("quantize", L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot, gm,
+                                                          p["codes"], p["scales"], g, sh)))
+                seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
+                                                            fmt, block, rot, p["bm"], p["terms"], p["ws"],
+                                                            b["ws"].numel(), sh)))
+            else:
+                seq.append(("quantize_mse", L.fp4q_quantize_mse,
+                            (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], g, p["bm"],
+                             p["terms"], p["ws"], b["ws"].numel(), sh)))
             seq.append(("dequantize", L.fp4q_dequantize, (p["codes"], p["scales"], g, rows, cols, fmt, block, 0,
                                                           0, p["deq"], sh)))
-            seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols, fmt,
-                                                        block, rot, p["bm"], p["terms"], p["ws"],
-                                                        b["ws"].numel(), sh)))
             self.calls.append(seq)
         self.elements = sum(x.numel() for _, x, *_ in items)
-        # kernels per step: amax + G (per-tensor scale), quantize, dequantize, MSE + its finalize
-        self.launches_per_step = sum(4 + (2 if gm == COMP else 0) for *_, gm in items)
+        # kernels per step: amax + G (per-tensor scale), quantize (+MSE) and the MSE finalize, dequantize
+        self.launches_per_step = sum(3 + (2 if gm == COMP else 0) + (1 if separate_mse else 0)
+                                     for *_, gm in items)
         self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
 
     def step(self, stream, ev=None):
@@ -392,7 +400,7 @@ def main(argv=None):
     items = build_workload(args.workload, device, rank, args)
     stream = torch.cuda.Stream(device)
     stream.wait_stream(torch.cuda.current_stream())
-    pipe = Pipeline(fq, items, device, stream)
+    pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse)
     in_l2 = sum(x.numel() * 2 for _, x, *_ in items) < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
 

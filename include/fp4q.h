@@ -156,7 +156,23 @@ FP4Q_API int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* 
                    float* block_mse, double* terms, void* workspace, size_t ws_bytes,
                    void* stream);
 
-/* Bytes of device workspace fp4q_block_mse needs for this shape (host only). */
+/*
+ * fp4q_quantize_mse -- fp4q_quantize and the MSE of fp4q_block_mse in one pass
+ * over x: the errors are measured in the quantizing kernel, from the values
+ * and codes it has in registers, so x is read once instead of twice.  Outputs
+ * and arguments as for the two calls; block_mse may be NULL.  The block
+ * maximum's error is taken against the largest dequantized magnitude of the
+ * block (the value the maximum rounds to), the per-block sums are fp32 and the
+ * tensor terms fp64 in a fixed order.  workspace: at least
+ * fp4q_block_mse_workspace_size() bytes.
+ */
+FP4Q_API int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                               int gmode, uint8_t* codes, uint8_t* scales, float* gscale,
+                               float* block_mse, double* terms, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* Bytes of device workspace fp4q_block_mse and fp4q_quantize_mse need for this
+ * shape (host only; at most 128 KiB). */
 FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block);
 
 /*

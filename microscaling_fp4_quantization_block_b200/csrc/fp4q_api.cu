@@ -113,7 +113,54 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
     p.scales = scales;
     p.gsrc = (gmode == FP4Q_GLOBAL_NONE) ? nullptr : gscale;
     rotation_constants(rot, &p.c_hi, &p.c_lo);
-    return cuda_status(launch_quantize(fmt, block, rot, p, s));
+    return cuda_status(launch_quantize(fmt, block, rot, false, p, nullptr, s));
+}
+
+int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                      uint8_t* codes, uint8_t* scales, float* gscale, float* block_mse, double* terms,
+                      void* workspace, size_t ws_bytes, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (gmode != FP4Q_GLOBAL_NONE && gmode != FP4Q_GLOBAL_COMPUTE && gmode != FP4Q_GLOBAL_GIVEN)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
+    if (gmode != FP4Q_GLOBAL_NONE) {
+        if (!gscale) return FP4Q_ERR_NULL;
+        if (!aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    }
+    if (!terms || !workspace) return FP4Q_ERR_NULL;
+    if (!aligned(terms, 8) || !aligned(workspace, 8)) return FP4Q_ERR_ALIGN;
+    if (n > 0) {
+        if (!x || !codes || !scales) return FP4Q_ERR_NULL;
+        if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)) return FP4Q_ERR_ALIGN;
+    }
+    if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
+    if (ws_bytes < fp4q_block_mse_workspace_size(rows, cols, block)) return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    if (gmode == FP4Q_GLOBAL_COMPUTE) {
+        cudaError_t e = enqueue_amax(x, n, rot, gscale, s);
+        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+        global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
+        if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    double* partials = static_cast<double*>(workspace);
+    int grid = 0;
+    if (n > 0) {
+        QuantParams p{};
+        p.x = static_cast<const uint16_t*>(x);
+        p.n = n;
+        p.codes = codes;
+        p.scales = scales;
+        p.gsrc = (gmode == FP4Q_GLOBAL_NONE) ? nullptr : gscale;
+        p.block_mse = block_mse;
+        p.partials = partials;
+        rotation_constants(rot, &p.c_hi, &p.c_lo);
+        if (launch_quantize(fmt, block, rot, true, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
+    return cuda_status(cudaGetLastError());
 }
 
 int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)
@@ -160,12 +207,8 @@ size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block)
 {
     (void)block;
     if (rows < 0 || cols < 0) return 0;
-    const int64_t n = rows * cols;
-    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
-    int64_t ctas = (tiles + kThreads / 32 - 1) / (kThreads / 32);
-    if (ctas < 1) ctas = 1;
-    if (ctas > kMaxMseCtas) ctas = kMaxMseCtas;
-    return (size_t)ctas * 4 * sizeof(double);
+    if (cols != 0 && rows > INT64_MAX / 4 / cols) return 0;
+    return (size_t)partial_slots(rows * cols) * 4 * sizeof(double);
 }
 
 int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, const float* gscale,
@@ -187,8 +230,6 @@ int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, c
     double* partials = static_cast<double*>(workspace);
     int grid = 0;
     if (n > 0) {
-        grid = mse_grid(block, rot, n);
-        if (grid <= 0) return FP4Q_ERR_UNSUPPORTED;
         MseParams p{};
         p.x = static_cast<const uint16_t*>(x);
         p.codes = codes;
@@ -199,7 +240,7 @@ int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, c
         p.block_mse = block_mse;
         p.partials = partials;
         rotation_constants(rot, &p.c_hi, &p.c_lo);
-        if (launch_block_mse(block, rot, p, grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+        if (launch_block_mse(block, rot, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
     }
     mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
     return cuda_status(cudaGetLastError());
@@ -212,7 +253,7 @@ int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* strea
     if (!r || !packed) return FP4Q_ERR_NULL;
     if (!aligned(r, 4) || !aligned(packed, 4)) return FP4Q_ERR_ALIGN;
     const int64_t work = (n + 7) / 8;
-    int grid = resident_grid((const void*)e2m1_encode_kernel, (work + kThreads - 1) / kThreads);
+    int grid = grid_for((const void*)e2m1_encode_kernel, 0, (work + kThreads - 1) / kThreads);
     e2m1_encode_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(r, n, packed);
     return cuda_status(cudaGetLastError());
 }
@@ -225,7 +266,7 @@ int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, vo
     if (n == 0) return FP4Q_OK;
     if (!s || !codes) return FP4Q_ERR_NULL;
     if (!aligned(s, 4) || !aligned(codes, 4)) return FP4Q_ERR_ALIGN;
-    int grid = resident_grid((const void*)scale_encode_kernel, (n + kThreads - 1) / kThreads);
+    int grid = grid_for((const void*)scale_encode_kernel, 0, (n + kThreads - 1) / kThreads);
     scale_encode_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(s, n, fmt, codes);
     return cuda_status(cudaGetLastError());
 }

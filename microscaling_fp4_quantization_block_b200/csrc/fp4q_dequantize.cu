@@ -9,9 +9,10 @@ template <int B, int K, bool F32>
 cudaError_t run_dequantize(const DequantParams& p, cudaStream_t s)
 {
     auto kern = dequantize_kernel<B, K, F32>;
-    const int64_t tiles = (p.n + kTileElems - 1) / kTileElems;
-    const int grid = resident_grid((const void*)kern, (tiles + kThreads / 32 - 1) / (kThreads / 32));
-    kern<<<grid, kThreads, 0, s>>>(p);
+    const int64_t tile_elems = 32 * DPL;  // 32 lanes x 128 elements
+    const int64_t tiles = (p.n + tile_elems - 1) / tile_elems;
+    const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
+    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -22,15 +23,14 @@ cudaError_t deq_out(bool f32, const DequantParams& p, cudaStream_t s)
 }
 
 template <int B, int K>
-const void* mse_kernel_ptr()
+cudaError_t run_mse(const MseParams& p, int* grid_out, cudaStream_t s)
 {
-    return (const void*)block_mse_kernel<B, K>;
-}
-
-template <int B, int K>
-cudaError_t run_mse(const MseParams& p, int grid, cudaStream_t s)
-{
-    block_mse_kernel<B, K><<<grid, kThreads, 0, s>>>(p);
+    auto kern = block_mse_kernel<B, K>;
+    int64_t need = ring_ctas_needed(p.n, EPT);
+    if (need > partial_slots(p.n)) need = partial_slots(p.n);
+    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
+    *grid_out = grid;
+    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -64,20 +64,9 @@ cudaError_t launch_dequantize(int B, int K, bool f32out, const DequantParams& p,
     return cudaErrorInvalidValue;
 }
 
-int mse_grid(int B, int K, int64_t n)
+cudaError_t launch_block_mse(int B, int K, const MseParams& p, int* grid_out, cudaStream_t s)
 {
-    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
-    int64_t need = (tiles + kThreads / 32 - 1) / (kThreads / 32);
-    if (need > kMaxMseCtas) need = kMaxMseCtas;
-#define MSE_PTR(BB, KK) return resident_grid(mse_kernel_ptr<BB, KK>(), need);
-    FP4Q_BK_SWITCH(B, K, MSE_PTR)
-#undef MSE_PTR
-    return 0;
-}
-
-cudaError_t launch_block_mse(int B, int K, const MseParams& p, int grid, cudaStream_t s)
-{
-#define MSE_CALL(BB, KK) return run_mse<BB, KK>(p, grid, s);
+#define MSE_CALL(BB, KK) return run_mse<BB, KK>(p, grid_out, s);
     FP4Q_BK_SWITCH(B, K, MSE_CALL)
 #undef MSE_CALL
     return cudaErrorInvalidValue;

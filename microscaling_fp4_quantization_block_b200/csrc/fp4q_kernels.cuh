@@ -2,15 +2,26 @@
 //
 // Every kernel treats the [rows][cols] tensor as one flat run of n elements:
 // blocks (block | cols) and rotation runs (rot | cols) never cross a row, so a
-// block is simply `block` consecutive elements of the flat run.  A thread owns
-// "units" of EPT consecutive elements (EPT = 16 or 32: one or two 256-bit
-// loads), the 32 lanes of a warp own 32 consecutive units, and a warp keeps
-// UNITS units per lane in flight (128 bytes of bf16 per lane) before it
-// computes, walking the tensor in a grid-stride loop whose trip count is the
-// same for every lane (lanes past the end hold zeros), so shuffles always see
-// the full warp.  A block wider than a unit spans B/EPT adjacent lanes, whose
-// maximum is combined with shuffles; a rotation run wider than a unit is
-// finished with butterfly stages across K/EPT adjacent lanes.
+// block is simply `block` consecutive elements of the flat run.
+//
+// Work decomposition.  A lane owns "units" of 32 consecutive elements; the 32
+// lanes of a warp own the 32 consecutive units of a 1024-element "tile"
+// (quantize, amax, MSE), so blocks of 8, 16 or 32 sit inside one lane, wider
+// blocks and rotation runs span adjacent lanes (maxima combined with
+// shuffles, butterflies finished across lanes).  Warps walk tiles in a
+// grid-stride loop with the same trip count for every lane (lanes past the
+// end hold zeros), so shuffles always see the whole warp.
+//
+// Memory pipeline.  The streamed input goes through a per-warp ring of
+// NSTAGE tiles in shared memory filled with 16-byte cp.async copies: while a
+// warp computes tile i, tiles i+1 .. i+NSTAGE-1 are in flight (6 KB per warp),
+// independent of the compute.  Each copy instruction moves 512 contiguous
+// bytes per warp; chunks land XOR-swizzled so each lane reads its own unit
+// back with conflict-free 128-bit shared loads.
+//
+// Arithmetic.  Element values live as fp32 pairs (f32x2) so that products,
+// sums and butterflies issue as packed two-wide instructions; the scales of
+// two blocks are computed together the same way.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -20,85 +31,318 @@
 namespace fp4q {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRingBytesPerWarp = 8192;
+constexpr int kRingBytesPerCta = kRingBytesPerWarp * kWarps;
+constexpr int EPT = 32;                                          // elements per unit
 
 template <int B, int K>
 struct UnitShape {
-    static constexpr int kMaxBK = (B > K ? B : K);
-    static constexpr int EPT = kMaxBK <= 16 ? 16 : 32;           // elements per unit
-    static constexpr int UNITS = EPT == 16 ? 4 : 2;              // units in flight per lane
-    static constexpr int kBlocksPerUnit = B <= EPT ? EPT / B : 1;
-    static constexpr int kLanesPerBlock = B <= EPT ? 1 : B / EPT;
-    static constexpr int kChunk = K == 0 ? 1 : (K <= EPT ? K : EPT); // in-register run
+    static constexpr int NB = B <= EPT ? EPT / B : 1;             // blocks per unit
+    static constexpr int LPB = B <= EPT ? 1 : B / EPT;            // lanes per block
+    static constexpr int BE = B <= EPT ? B : EPT;                 // elements of a block in one unit
+    static constexpr int kChunk = K == 0 ? 1 : (K <= EPT ? K : EPT); // in-register rotation run
     static constexpr int kRotLanes = K > EPT ? K / EPT : 1;
-    static constexpr int kBlockElems = B <= EPT ? B : EPT;        // elements of a block in one unit
-    static_assert(kLanesPerBlock <= 32 && kRotLanes <= 32, "block or rotation wider than a warp");
+    static_assert(LPB <= 32 && kRotLanes <= 32, "block or rotation wider than a warp");
 };
 
-// ---------------------------------------------------------------- unit loads
-// Raw bf16 words of one unit (word k = elements 2k, 2k+1).  A unit that runs
-// past n (only the last one) is read element by element and zero-padded; the
-// padding occupies whole blocks and rotation runs because n is a multiple of
-// both, so it never mixes with real data.
-template <int EPT>
-__device__ __forceinline__ void load_unit(const uint16_t* __restrict__ x, int64_t n, int64_t u,
-                                          uint32_t (&w)[EPT / 2])
-{
-    const int64_t e0 = u * EPT;
-    if (e0 + EPT <= n) {
+// ---------------------------------------------------------------- ring of tiles
+// BYTES_PER_UNIT bytes of input per unit (16, 32 or 64), UPS units per lane
+// per tile.  All per-lane offsets are computed once; a tile that lies wholly
+// inside the input is copied with one cp.async per 16-byte chunk at immediate
+// offsets, only the last tile of the input takes the clamped path.
+template <int BYTES_PER_UNIT, int UPS>
+struct Ring {
+    static constexpr int CPL = BYTES_PER_UNIT / 16;               // 16-byte chunks per lane per sub-tile
+    static constexpr int SUB_BYTES = 32 * BYTES_PER_UNIT;         // one sub-tile
+    static constexpr int TILE_BYTES = UPS * SUB_BYTES;
+    static constexpr int NSTAGE = kRingBytesPerWarp / TILE_BYTES;
+    static_assert(NSTAGE >= 2, "ring too small");
+    static_assert(CPL == 1 || CPL == 2 || CPL == 4, "unsupported unit size");
+
+    uint32_t base;                 // shared address of this warp's ring
+    uint32_t wr[CPL];              // shared offset (in a sub-tile) of the chunk this lane copies, per c
+    uint32_t rd[CPL];              // shared offset (in a sub-tile) of this lane's c-th chunk
+
+    // smem chunk of global chunk j of a sub-tile: XOR swizzle that keeps both
+    // the contiguous copies and the per-lane 128-bit reads conflict free.
+    static __device__ __forceinline__ int swz(int j) { return CPL == 1 ? j : (j ^ ((j >> 3) & (CPL - 1))); }
+
+    __device__ __forceinline__ Ring(uint32_t b, int lane) : base(b)
+    {
 #pragma unroll
-        for (int h = 0; h < EPT / 16; ++h) {
-            U32x8 r = ldg256_stream(x + e0 + 16 * h);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) w[8 * h + k] = r.v[k];
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < EPT / 2; ++k) {
-            uint32_t lo = (e0 + 2 * k < n) ? (uint32_t)x[e0 + 2 * k] : 0u;
-            uint32_t hi = (e0 + 2 * k + 1 < n) ? (uint32_t)x[e0 + 2 * k + 1] : 0u;
-            w[k] = lo | (hi << 16);
+        for (int c = 0; c < CPL; ++c) {
+            wr[c] = 16u * (uint32_t)swz(lane + 32 * c);
+            rd[c] = 16u * (uint32_t)swz(CPL * lane + c);
         }
     }
+
+    // Start the copies of the tile at byte offset off of src (nbytes long in
+    // all) into stage s.  Bytes at or past nbytes are never read: a chunk
+    // that straddles the end copies its valid prefix, and the rest, like every
+    // chunk past the end, is zero-filled.
+    __device__ __forceinline__ void issue(const uint8_t* __restrict__ src, int64_t nbytes, int64_t off, int s,
+                                          int lane) const
+    {
+        const uint32_t sb = base + (uint32_t)(s * TILE_BYTES);
+        const uint8_t* g = src + off + 16 * lane;
+        if (off + TILE_BYTES <= nbytes) {
+#pragma unroll
+            for (int h = 0; h < UPS; ++h)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    cp_async16(sb + (uint32_t)(h * SUB_BYTES) + wr[c], g + h * SUB_BYTES + 512 * c, 16u);
+        } else {
+#pragma unroll
+            for (int h = 0; h < UPS; ++h)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    const int64_t o = off + h * SUB_BYTES + 512 * c + 16 * lane;
+                    const int64_t left = nbytes - o;
+                    const uint32_t cnt = left >= 16 ? 16u : (left > 0 ? (uint32_t)left : 0u);
+                    cp_async16(sb + (uint32_t)(h * SUB_BYTES) + wr[c], cnt ? (const void*)(src + o) : (const void*)src,
+                               cnt);
+                }
+        }
+    }
+
+    // This lane's unit of sub-tile h of stage s, as 32-bit words.
+    __device__ __forceinline__ void read(int s, int h, uint32_t (&w)[BYTES_PER_UNIT / 4]) const
+    {
+        const uint32_t sb = base + (uint32_t)(s * TILE_BYTES + h * SUB_BYTES);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const uint4 v = lds128(sb + rd[c]);
+            w[4 * c + 0] = v.x;
+            w[4 * c + 1] = v.y;
+            w[4 * c + 2] = v.z;
+            w[4 * c + 3] = v.w;
+        }
+    }
+};
+
+template <typename R>
+__device__ __forceinline__ R warp_ring(uint8_t* smem)
+{
+    return R((uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)((threadIdx.x >> 5) * kRingBytesPerWarp),
+             threadIdx.x & 31);
 }
 
-template <int EPT>
-__device__ __forceinline__ void unpack_unit(const uint32_t (&w)[EPT / 2], float (&v)[EPT])
+// Ring pipeline driver: calls body(tile, stage) for every tile of this warp,
+// with the tile's input resident in the ring.  NSTAGE - 1 tiles are in flight.
+template <typename R, typename Body>
+__device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __restrict__ src, int64_t nbytes,
+                                             int64_t n_tiles, int64_t warp, int64_t n_warps, int lane,
+                                             Body&& body)
+{
+    constexpr int NS = R::NSTAGE;
+    const int64_t step = n_warps * R::TILE_BYTES;
+    int64_t t_issue = warp;
+    int64_t off_issue = warp * R::TILE_BYTES;
+#pragma unroll
+    for (int s = 0; s < NS - 1; ++s) {
+        if (t_issue < n_tiles) ring.issue(src, nbytes, off_issue, s, lane);
+        cp_async_commit();
+        t_issue += n_warps;
+        off_issue += step;
+    }
+    int stage = 0;
+    for (int64_t t = warp; t < n_tiles; t += n_warps) {
+        const int s_new = stage == 0 ? NS - 1 : stage - 1;          // the slot read last iteration
+        if (t_issue < n_tiles) ring.issue(src, nbytes, off_issue, s_new, lane);
+        cp_async_commit();
+        t_issue += n_warps;
+        off_issue += step;
+        cp_async_wait<NS - 1>();                                   // tile t has landed (own copies)
+        __syncwarp();                                              // ... and every lane's copies
+        body(t, stage);
+        stage = stage + 1 == NS ? 0 : stage + 1;
+        __syncwarp();                                              // slot may be refilled next iteration
+    }
+    cp_async_wait_all();
+}
+
+using XRing = Ring<2 * EPT, 1>;                                  // one bf16 unit per lane per tile
+
+// bf16 words -> fp32 pairs (exact widening).
+__device__ __forceinline__ void unpack_unit(const uint32_t (&w)[EPT / 2], f32x2 (&p)[EPT / 2])
 {
 #pragma unroll
-    for (int k = 0; k < EPT / 2; ++k) {
-        v[2 * k] = bf16_lo(w[k]);
-        v[2 * k + 1] = bf16_hi(w[k]);
-    }
+    for (int k = 0; k < EPT / 2; ++k) p[k] = pk(bf16_lo(w[k]), bf16_hi(w[k]));
 }
 
 // Optional rotation of a unit held in registers: runs of K elements, the part
 // inside the unit in registers, the rest across lanes, then 1/sqrt(K).
-template <int B, int K>
-__device__ __forceinline__ void rotate_unit(float (&v)[UnitShape<B, K>::EPT], int lane, float c_hi,
-                                            float c_lo)
+template <int K>
+__device__ __forceinline__ void rotate_unit(f32x2 (&p)[EPT / 2], int lane, float c_hi, float c_lo)
 {
-    using S = UnitShape<B, K>;
     if constexpr (K > 0) {
-        fwht_inreg<S::EPT, S::kChunk>(v);
-        if constexpr (S::kRotLanes > 1) fwht_xlane<S::EPT, S::kRotLanes>(v, lane);
-        normalize<S::EPT>(v, c_hi, c_lo);
+        fwht_inreg<EPT, (K < EPT ? K : EPT)>(p);
+        if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(p, lane);
+        normalize<EPT>(p, c_hi, c_lo);
     }
+}
+
+// Absolute maximum of the CNT values of p (CNT even).
+template <int CNT>
+__device__ __forceinline__ float pairs_absmax(const f32x2* p)
+{
+    float a, b, m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < CNT / 2; ++k) {
+        upk(p[k], a, b);
+        m = amax3(a, b, m);
+    }
+    return m;
 }
 
 // Per-block absolute maximum of a unit (combined across lanes for wide blocks).
 template <int B, int K>
-__device__ __forceinline__ void block_max(const float (&v)[UnitShape<B, K>::EPT],
-                                          float (&m)[UnitShape<B, K>::kBlocksPerUnit])
+__device__ __forceinline__ void block_max(const f32x2 (&p)[EPT / 2], float (&m)[UnitShape<B, K>::NB])
 {
     using S = UnitShape<B, K>;
 #pragma unroll
-    for (int bi = 0; bi < S::kBlocksPerUnit; ++bi) {
-        float a = 0.0f;
+    for (int bi = 0; bi < S::NB; ++bi) m[bi] = pairs_absmax<S::BE>(p + bi * S::BE / 2);
+    if constexpr (S::LPB > 1) m[0] = group_max<S::LPB>(m[0]);
+}
+
+template <int LANES>
+__device__ __forceinline__ float group_sum(float s)
+{
 #pragma unroll
-        for (int i = 0; i < S::kBlockElems; ++i) a = fmaxf(a, fabsf(v[bi * S::kBlockElems + i]));
-        m[bi] = a;
+    for (int d = 1; d < LANES; d <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, d));
+    return s;
+}
+
+// Per-CTA reduction of four fp64 accumulators into partials[blockIdx.x][4], in a
+// fixed order (warp butterflies, then warps in index order): deterministic.
+__device__ __forceinline__ void cta_partials(double a0, double a1, double a2, double a3, double* partials)
+{
+    __shared__ double red[kWarps][4];
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, d);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, d);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, d);
+        a3 += __shfl_xor_sync(0xffffffffu, a3, d);
     }
-    if constexpr (S::kLanesPerBlock > 1) m[0] = group_max<S::kLanesPerBlock>(m[0]);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0) {
+        red[wid][0] = a0;
+        red[wid][1] = a1;
+        red[wid][2] = a2;
+        red[wid][3] = a3;
+    }
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        double s = 0.0;
+        for (int k = 0; k < kWarps; ++k) s += red[k][threadIdx.x];
+        partials[(int64_t)blockIdx.x * 4 + threadIdx.x] = s;
+    }
+}
+
+// Grid values of the 8 nibbles of a code word as 4 fp32 pairs (exact).
+__device__ __forceinline__ void decode8(uint32_t cw, f32x2 (&g)[4])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a, b;
+        e2m1_unpack2((cw >> (8 * j)) & 0xffu, a, b);
+        g[j] = pk(a, b);
+    }
+}
+
+// E2M1 codes of 4 pairs -> one code word (low nibble = even element).
+__device__ __forceinline__ uint32_t pack_pairs(f32x2 p0, f32x2 p1, f32x2 p2, f32x2 p3)
+{
+    float a0, b0, a1, b1, a2, b2, a3, b3;
+    upk(p0, a0, b0);
+    upk(p1, a1, b1);
+    upk(p2, a2, b2);
+    upk(p3, a3, b3);
+    return e2m1_pack8(a0, b0, a1, b1, a2, b2, a3, b3);
+}
+
+// Codes of 4 pairs with correctly rounded quotients v / s (s != 0): the rare
+// fallback of the bracketed element rounding, kept out of line.
+static __device__ __noinline__ uint32_t pack_pairs_div(f32x2 p0, f32x2 p1, f32x2 p2, f32x2 p3, float s)
+{
+    float a[8];
+    upk(p0, a[0], a[1]);
+    upk(p1, a[2], a[3]);
+    upk(p2, a[4], a[5]);
+    upk(p3, a[6], a[7]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = __fdiv_rn(a[j], s);
+    return e2m1_pack8(a[0], a[1], a[2], a[3], a[4], a[5], a[6], a[7]);
+}
+
+// Exact codes of 8 elements whose bracketed codes a (low end) and b (high end)
+// differ in some nibble: a quotient that sits at, or within 2^-18 of, an E2M1
+// rounding threshold t.  For such an element |y| and t S agree to ~8 bits, so
+// r = |y| - t S is exact through one fused multiply-add, and the correctly
+// rounded quotient fp32(|y| / S) equals t exactly when -h_lo S <= r <= h_hi S,
+// h being half the fp32 spacing below / above t (powers of two, so h S is
+// exact).  Then: r above the band -> the upper code, below -> the lower code,
+// inside -> the even one of the two (round half to even).  Elements whose two
+// codes agree keep them.  Kept out of line: it runs for ~0.1% of the words of
+// bf16 data whose per-tensor scale makes quotients land on thresholds.
+static __device__ __noinline__ uint32_t resolve_ties(uint32_t a, uint32_t b, f32x2 p0, f32x2 p1, f32x2 p2,
+                                                     f32x2 p3, float S)
+{
+    float y[8];
+    upk(p0, y[0], y[1]);
+    upk(p1, y[2], y[3]);
+    upk(p2, y[4], y[5]);
+    upk(p3, y[6], y[7]);
+    f32x2 gl[4], gh[4];
+    decode8(a, gl);
+    decode8(b, gh);
+    uint32_t out = a;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t ca = (a >> (4 * j)) & 0xfu, cb = (b >> (4 * j)) & 0xfu;
+        if (ca == cb) continue;
+        float la, lb, ha, hb;
+        upk(gl[j / 2], la, lb);
+        upk(gh[j / 2], ha, hb);
+        const float glo = fabsf((j & 1) ? lb : la), ghi = fabsf((j & 1) ? hb : ha);
+        const float t = __fmul_rn(__fadd_rn(glo, ghi), 0.5f);            // the threshold between them
+        const uint32_t tb = __float_as_uint(t);
+        const float hu = __uint_as_float((tb & 0x7f800000u) - (24u << 23)); // half spacing above t
+        const float hl = (tb & 0x007fffffu) ? hu : __fmul_rn(hu, 0.5f);     // ... below t
+        const float r = __fmaf_rn(-t, S, fabsf(y[j]));
+        uint32_t mag;
+        if (r > __fmul_rn(hu, S)) mag = cb & 7u;
+        else if (r < -__fmul_rn(hl, S)) mag = ca & 7u;
+        else mag = ((ca & 7u) & 1u) ? (cb & 7u) : (ca & 7u);              // tie: even magnitude code
+        out = (out & ~(0xfu << (4 * j))) | (((ca & 8u) | mag) << (4 * j));
+    }
+    return out;
+}
+
+// Scales of the NB blocks of a unit: codes, S and the bracket of 1/S.  The UE4M3
+// rule runs on two blocks at a time with two-wide instructions.
+template <int FMT, int NB>
+__device__ __forceinline__ bool unit_scales(const float (&m)[NB], const ScaleConsts& kc, uint32_t (&code)[NB],
+                                            float (&S)[NB], float (&rlo)[NB], float (&rhi)[NB])
+{
+    bool exact = true;
+    if constexpr (FMT == kUE4M3 && NB >= 2) {
+#pragma unroll
+        for (int bi = 0; bi < NB; bi += 2) {
+            exact = block_scale_ue4m3_pair(m[bi], m[bi + 1], kc, code[bi], code[bi + 1], S[bi], S[bi + 1], rlo[bi],
+                                           rlo[bi + 1], rhi[bi], rhi[bi + 1]) && exact;
+        }
+    } else {
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) {
+            bool ok;
+            code[bi] = block_scale<FMT>(m[bi], kc, S[bi], rlo[bi], rhi[bi], ok);
+            exact = exact && ok;
+        }
+    }
+    return exact;
 }
 
 // ---------------------------------------------------------------- quantize
@@ -109,82 +353,106 @@ struct QuantParams {
     uint8_t* scales;       // n/B bytes
     const float* gsrc;     // per-tensor scale G (nullptr: G = 1)
     float c_hi, c_lo;      // 1/sqrt(K) split in two fp32 parts
+    float* block_mse;      // fused MSE: n/B floats or nullptr
+    double* partials;      // fused MSE: [gridDim.x][4]
 };
 
-template <int FMT, int B, int K>
-__device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[UnitShape<B, K>::EPT / 2],
-                                              int lane, float G, float denom)
+template <int FMT, int B, int K, bool MSE>
+__device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
+                                              int lane, const ScaleConsts& kc, double (&acc)[4])
 {
     using S = UnitShape<B, K>;
-    constexpr int EPT = S::EPT;
-    constexpr int NB = S::kBlocksPerUnit;
-    float v[EPT];
-    unpack_unit<EPT>(w, v);
-    rotate_unit<B, K>(v, lane, p.c_hi, p.c_lo);
+    constexpr int NB = S::NB, BE = S::BE;
+    f32x2 v[EPT / 2];
+    unpack_unit(w, v);
+    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
 
     float m[NB];
     block_max<B, K>(v, m);
 
-    float sc[NB], rc[NB];
+    float sc[NB], rlo[NB], rhi[NB];
     uint32_t code[NB];
-    bool slow_scale = false;
-#pragma unroll
-    for (int bi = 0; bi < NB; ++bi) {
-        code[bi] = block_scale<FMT>(m[bi], G, denom, sc[bi], rc[bi]);
-        if constexpr (FMT != kE8M0) {
-            if (sc[bi] == 0.0f) rc[bi] = 0.0f;                       // zero-rounded block
-            else if (!scale_product_safe(sc[bi])) slow_scale = true;
-        }
-    }
+    const bool exact = unit_scales<FMT, NB>(m, kc, code, sc, rlo, rhi);
 
     uint32_t cw[EPT / 8];
     if constexpr (FMT == kE8M0) {
-        // S is a power of two: y * (1/S) is exact, so it is the quotient itself.
+        // S is a power of two: y * (1/S) is exactly the quotient.
 #pragma unroll
         for (int k = 0; k < EPT / 8; ++k) {
-            float q[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = 8 * k + j;
-                q[j] = __fmul_rn(v[i], rc[i / S::kBlockElems]);
-            }
-            cw[k] = e2m1_pack8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+            const f32x2 r = pk(rlo[(8 * k) / BE], rlo[(8 * k) / BE]);
+            cw[k] = pack_pairs(mul2(v[4 * k], r), mul2(v[4 * k + 1], r), mul2(v[4 * k + 2], r),
+                               mul2(v[4 * k + 3], r));
         }
     } else {
-        bool agree = !slow_scale;
 #pragma unroll
         for (int k = 0; k < EPT / 8; ++k) {
-            float lo[8], hi[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = 8 * k + j;
-                const float q0 = __fmul_rn(v[i], rc[i / S::kBlockElems]);
-                lo[j] = __fmul_rn(q0, kBracketLo);
-                hi[j] = __fmul_rn(q0, kBracketHi);
-            }
-            const uint32_t a = e2m1_pack8(lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
-            const uint32_t b = e2m1_pack8(hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
-            agree = agree && (a == b);
-            cw[k] = a;
+            const int bi = (8 * k) / BE;
+            const f32x2 rl = pk(rlo[bi], rlo[bi]), rh = pk(rhi[bi], rhi[bi]);
+            const uint32_t a = pack_pairs(mul2(v[4 * k], rl), mul2(v[4 * k + 1], rl), mul2(v[4 * k + 2], rl),
+                                          mul2(v[4 * k + 3], rl));
+            const uint32_t b = pack_pairs(mul2(v[4 * k], rh), mul2(v[4 * k + 1], rh), mul2(v[4 * k + 2], rh),
+                                          mul2(v[4 * k + 3], rh));
+            // a quotient on (or within the bracket of) a threshold: settle it exactly
+            cw[k] = (a == b) ? a : resolve_ties(a, b, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], sc[bi]);
         }
-        if (!agree) {
-            // rare: a quotient near an E2M1 rounding threshold, or an extreme scale
+        if (!exact) {
+            // extreme scales (S or 1/S not a normal float): correctly rounded divisions
 #pragma unroll
             for (int k = 0; k < EPT / 8; ++k) {
-                float q[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = 8 * k + j;
-                    const float s = sc[i / S::kBlockElems];
-                    q[j] = s != 0.0f ? __fdiv_rn(v[i], s) : 0.0f;
-                }
-                cw[k] = e2m1_pack8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+                const float s = sc[(8 * k) / BE];
+                if (s != 0.0f) cw[k] = pack_pairs_div(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], s);
             }
         }
         // zero-rounded blocks store plain 0x0 nibbles
 #pragma unroll
         for (int k = 0; k < EPT / 8; ++k)
-            if (sc[(8 * k) / S::kBlockElems] == 0.0f) cw[k] = 0u;
+            if (sc[(8 * k) / BE] == 0.0f) cw[k] = 0u;
+    }
+
+    // ---- fused MSE (three-term split of "Finer is better?"): v_i = decode(code_i) * S
+    if constexpr (MSE) {
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) {
+            const f32x2 s2 = pk(sc[bi], sc[bi]);
+            f32x2 sum = pk(0.0f, 0.0f);
+            float vmax = 0.0f;
+#pragma unroll
+            for (int k = bi * BE / 8; k < (bi + 1) * BE / 8; ++k) {
+                f32x2 g[4];
+                decode8(cw[k], g);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const f32x2 d = sub2(v[4 * k + j], mul2_rounded(g[j], s2));   // y - fp32(g S)
+                    sum = fma2(d, d, sum);
+                    float a, b;
+                    upk(g[j], a, b);
+                    vmax = amax3(a, b, vmax);
+                }
+            }
+            vmax = __fmul_rn(vmax, sc[bi]);                          // largest |v| of the block
+            float se, so;
+            upk(sum, se, so);
+            float s = __fadd_rn(se, so);
+            if constexpr (S::LPB > 1) {
+                s = group_sum<S::LPB>(s);
+                vmax = group_max<S::LPB>(vmax);
+            }
+            const int64_t eb = u * EPT + (int64_t)bi * BE;
+            const bool leader = (S::LPB == 1) || ((lane % S::LPB) == 0);
+            if (leader && eb < p.n) {
+                if (p.block_mse) p.block_mse[eb / B] = __fmul_rn(s, 1.0f / (float)B);
+                acc[0] += (double)s;
+                if (vmax == 0.0f) {
+                    acc[3] += (double)s;
+                } else {
+                    // the block maximum rounds to the largest |v| of the block
+                    const float dm = __fsub_rn(m[bi], vmax);
+                    const float emax = __fmul_rn(dm, dm);
+                    acc[2] += (double)emax;
+                    acc[1] += (double)s - (double)emax;
+                }
+            }
+        }
     }
 
     // ---- stores
@@ -192,8 +460,7 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     if (e0 >= p.n) return;
     uint8_t* cdst = p.codes + e0 / 2;
     if (e0 + EPT <= p.n) {
-        if constexpr (EPT == 16) stg64(cdst, cw[0], cw[1]);
-        else stg128(cdst, cw[0], cw[1], cw[2], cw[3]);
+        stg128(cdst, cw[0], cw[1], cw[2], cw[3]);
     } else {
         const int nbytes = (int)((p.n - e0) / 2);
 #pragma unroll
@@ -202,8 +469,8 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
             for (int j = 0; j < 4; ++j)
                 if (4 * k + j < nbytes) cdst[4 * k + j] = (uint8_t)(cw[k] >> (8 * j));
     }
-    if constexpr (S::kLanesPerBlock > 1) {
-        if ((lane % S::kLanesPerBlock) == 0) p.scales[e0 / B] = (uint8_t)code[0];
+    if constexpr (S::LPB > 1) {
+        if ((lane % S::LPB) == 0) p.scales[e0 / B] = (uint8_t)code[0];
     } else {
         const int64_t b0 = e0 / B;
         const int64_t nblk = p.n / B;
@@ -212,12 +479,9 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
                 p.scales[b0] = (uint8_t)code[0];
             } else if constexpr (NB == 2) {
                 *reinterpret_cast<uint16_t*>(p.scales + b0) = (uint16_t)(code[0] | (code[1] << 8));
-            } else if constexpr (NB == 4) {
+            } else {
                 *reinterpret_cast<uint32_t*>(p.scales + b0) =
                     code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24);
-            } else {
-#pragma unroll
-                for (int bi = 0; bi < NB; ++bi) p.scales[b0 + bi] = (uint8_t)code[bi];
             }
         } else {
 #pragma unroll
@@ -227,34 +491,28 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     }
 }
 
-template <int FMT, int B, int K>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p)
+template <int FMT, int B, int K, bool MSE>
+__global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantParams p)
 {
-    using S = UnitShape<B, K>;
-    constexpr int EPT = S::EPT, U = S::UNITS;
+    extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
-    const int64_t n_units = (p.n + EPT - 1) / EPT;
-    const int64_t n_tiles = (n_units + 32 * U - 1) / (32 * U);
+    const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const XRing ring = warp_ring<XRing>(smem_ring);
 
     float G = 1.0f;
     if (FMT != kE8M0 && p.gsrc != nullptr) G = *p.gsrc;
-    const float denom = __fmul_rn(6.0f, G);
+    const ScaleConsts kc = scale_consts(G);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
 
-    for (int64_t tile = warp; tile < n_tiles; tile += n_warps) {
-        uint32_t w[U][EPT / 2];
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            load_unit<EPT>(p.x, p.n, u, w[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            quantize_unit<FMT, B, K>(p, u, w[j], lane, G, denom);
-        }
-    }
+    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
+                 [&](int64_t t, int s) {
+                     uint32_t w[EPT / 2];
+                     ring.read(s, 0, w);
+                     quantize_unit<FMT, B, K, MSE>(p, t * 32 + lane, w, lane, kc, acc);
+                 });
+    if constexpr (MSE) cta_partials(acc[0], acc[1], acc[2], acc[3], p.partials);
 }
 
 // ---------------------------------------------------------------- per-tensor amax
@@ -268,27 +526,33 @@ struct AmaxParams {
 template <int K>
 __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
 {
-    using S = UnitShape<16, K>;
-    constexpr int EPT = S::EPT, U = S::UNITS;
+    extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
-    const int64_t n_units = (p.n + EPT - 1) / EPT;
-    const int64_t n_tiles = (n_units + 32 * U - 1) / (32 * U);
+    const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const XRing ring = warp_ring<XRing>(smem_ring);
     float mx = 0.0f;
-    for (int64_t tile = warp; tile < n_tiles; tile += n_warps) {
-        uint32_t w[U][EPT / 2];
+    uint32_t mb = 0;                                       // max |bf16| pattern, two halves
+    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
+                 [&](int64_t, int s) {
+                     uint32_t w[EPT / 2];
+                     ring.read(s, 0, w);
+                     if constexpr (K == 0) {
+                         // |bf16| patterns order like their values: SIMD max of both halves
 #pragma unroll
-        for (int j = 0; j < U; ++j) load_unit<EPT>(p.x, p.n, (tile * U + j) * 32 + lane, w[j]);
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-            float v[EPT];
-            unpack_unit<EPT>(w[j], v);
-            rotate_unit<16, K>(v, lane, p.c_hi, p.c_lo);
-#pragma unroll
-            for (int i = 0; i < EPT; ++i) mx = fmaxf(mx, fabsf(v[i]));
-        }
-    }
+                         for (int k = 0; k < EPT / 2; ++k) {
+                             const uint32_t a = w[k] & 0x7fff7fffu;
+                             asm("max.u16x2 %0, %0, %1;" : "+r"(mb) : "r"(a));
+                         }
+                     } else {
+                         f32x2 v[EPT / 2];
+                         unpack_unit(w, v);
+                         rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+                         mx = fmaxf(mx, pairs_absmax<EPT>(v));
+                     }
+                 });
+    if constexpr (K == 0) mx = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
     mx = group_max<32>(mx);
     if (lane == 0 && mx > 0.0f) atomicMax(p.amax_bits, __float_as_uint(mx));
 }
@@ -300,77 +564,12 @@ static __global__ void global_scale_kernel(const float* amax_in, float* gscale)
     *gscale = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
 }
 
-// ---------------------------------------------------------------- codes / scales of a unit
-template <int EPT>
-__device__ __forceinline__ void load_codes(const uint8_t* __restrict__ codes, int64_t n, int64_t u,
-                                           uint32_t (&cw)[EPT / 8])
+// Block scale from its code (decoded; G applied for the UE formats).
+__device__ __forceinline__ float decode_scale(uint32_t c, int fmt, float G)
 {
-    const int64_t e0 = u * EPT;
-    const uint8_t* src = codes + e0 / 2;
-    if (e0 + EPT <= n) {
-        if constexpr (EPT == 16) {
-            uint2 r = __ldg(reinterpret_cast<const uint2*>(src));
-            cw[0] = r.x;
-            cw[1] = r.y;
-        } else {
-            uint4 r = __ldg(reinterpret_cast<const uint4*>(src));
-            cw[0] = r.x;
-            cw[1] = r.y;
-            cw[2] = r.z;
-            cw[3] = r.w;
-        }
-    } else {
-        const int64_t nbytes = e0 < n ? (n - e0) / 2 : 0;
-#pragma unroll
-        for (int k = 0; k < EPT / 8; ++k) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (4 * k + j < nbytes) word |= (uint32_t)src[4 * k + j] << (8 * j);
-            cw[k] = word;
-        }
-    }
-}
-
-// Block scales S of a unit (decoded; G applied for the UE formats).
-template <int B, int K>
-__device__ __forceinline__ void load_scales(const uint8_t* __restrict__ scales, int fmt, float G,
-                                            int64_t n, int64_t u,
-                                            float (&S)[UnitShape<B, K>::kBlocksPerUnit])
-{
-    using Sh = UnitShape<B, K>;
-    const int64_t e0 = u * Sh::EPT;
-#pragma unroll
-    for (int bi = 0; bi < Sh::kBlocksPerUnit; ++bi) {
-        const int64_t e = e0 + (int64_t)bi * Sh::kBlockElems;
-        uint32_t c = e < n ? (uint32_t)__ldg(scales + e / B) : 0u;
-        float s;
-        if (fmt == kE8M0) s = e < n ? e8m0_decode(c) : 0.0f;
-        else if (fmt == kUE4M3) s = __fmul_rn(ue4m3_decode(c), G);
-        else s = __fmul_rn(ue5m3_decode(c), G);
-        S[bi] = s;
-    }
-}
-
-// Dequantized values of a unit: v = fp32(decode(nibble) * S).
-template <int B, int K>
-__device__ __forceinline__ void decode_unit(const uint32_t (&cw)[UnitShape<B, K>::EPT / 8],
-                                            const float (&S)[UnitShape<B, K>::kBlocksPerUnit],
-                                            float (&v)[UnitShape<B, K>::EPT])
-{
-    using Sh = UnitShape<B, K>;
-#pragma unroll
-    for (int k = 0; k < Sh::EPT / 8; ++k) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = 8 * k + 2 * j;
-            float lo, hi;
-            e2m1_unpack2((cw[k] >> (8 * j)) & 0xffu, lo, hi);
-            const float s = S[i / Sh::kBlockElems];
-            v[i] = __fmul_rn(lo, s);
-            v[i + 1] = __fmul_rn(hi, s);
-        }
-    }
+    if (fmt == kE8M0) return e8m0_decode(c);
+    if (fmt == kUE4M3) return __fmul_rn(ue4m3_decode(c), G);
+    return __fmul_rn(ue5m3_decode(c), G);
 }
 
 // ---------------------------------------------------------------- dequantize
@@ -384,66 +583,148 @@ struct DequantParams {
     float c_hi, c_lo;
 };
 
+// A lane owns DPL = 128 consecutive elements per tile: their 64 code bytes
+// stream through the ring, their DPL/B scale bytes are one vector load fetched
+// a tile ahead, and a rotation run of up to 128 elements stays in registers.
+constexpr int DPL = 128;
+
+template <int B>
+struct DeqScales {
+    static constexpr int NSB = B <= DPL ? DPL / B : 1;            // scale bytes per lane per tile
+    static constexpr int LPB = B <= DPL ? 1 : B / DPL;            // lanes per block
+};
+
+template <int B>
+__device__ __forceinline__ void fetch_scale_bytes(const uint8_t* __restrict__ scales, int64_t n, int64_t e0,
+                                                  uint32_t (&c)[DeqScales<B>::NSB])
+{
+    constexpr int NSB = DeqScales<B>::NSB;
+    const int64_t nblk = n / B;
+    const int64_t b0 = e0 / B;
+    if constexpr (NSB >= 4) {
+        if (b0 + NSB <= nblk) {
+            if constexpr (NSB == 4) {
+                const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(scales + b0));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) c[i] = (v >> (8 * i)) & 0xffu;
+            } else if constexpr (NSB == 8) {
+                const uint2 v = __ldg(reinterpret_cast<const uint2*>(scales + b0));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    c[i] = (v.x >> (8 * i)) & 0xffu;
+                    c[4 + i] = (v.y >> (8 * i)) & 0xffu;
+                }
+            } else {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(scales + b0));
+                const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < NSB; ++i) c[i] = (vv[i / 4] >> (8 * (i % 4))) & 0xffu;
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NSB; ++i) c[i] = (b0 + i < nblk) ? (uint32_t)__ldg(scales + b0 + i) : 0u;
+}
+
 template <int B, int K, bool F32OUT>
 __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
 {
-    using S = UnitShape<B, K>;
-    constexpr int EPT = S::EPT, U = S::UNITS;
+    constexpr int NSB = DeqScales<B>::NSB;
+    constexpr int EPB = B <= DPL ? B : DPL;                       // elements of a block in a lane
+    using R = Ring<64, 1>;                                        // 64 code bytes per lane per tile
+    extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
-    const int64_t n_units = (p.n + EPT - 1) / EPT;
-    const int64_t n_tiles = (n_units + 32 * U - 1) / (32 * U);
+    const int64_t n_tiles = (p.n + 32 * DPL - 1) / (32 * DPL);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const R ring = warp_ring<R>(smem_ring);
     const float G = (p.fmt != kE8M0 && p.gsrc != nullptr) ? *p.gsrc : 1.0f;
 
-    for (int64_t tile = warp; tile < n_tiles; tile += n_warps) {
-        uint32_t cw[U][EPT / 8];
-        float sc[U][S::kBlocksPerUnit];
+    uint32_t sc_next[NSB];
+    if (warp < n_tiles) fetch_scale_bytes<B>(p.scales, p.n, (warp * 32 + lane) * DPL, sc_next);
+
+    stream_tiles(ring, p.codes, p.n / 2, n_tiles, warp, n_warps, lane, [&](int64_t t, int s) {
+        const int64_t e0 = (t * 32 + lane) * DPL;
+        uint32_t scb[NSB];
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            load_codes<EPT>(p.codes, p.n, u, cw[j]);
-            load_scales<B, K>(p.scales, p.fmt, G, p.n, u, sc[j]);
-        }
+        for (int i = 0; i < NSB; ++i) scb[i] = sc_next[i];
+        if (t + n_warps < n_tiles) fetch_scale_bytes<B>(p.scales, p.n, ((t + n_warps) * 32 + lane) * DPL, sc_next);
+        uint32_t cw[16];
+        ring.read(s, 0, cw);
+        if (e0 >= p.n) return;
+        // chunks of CH elements: decode, rotate back (one run), round, store
+        constexpr int CH = K == 0 ? 16 : K;
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            float v[EPT];
-            decode_unit<B, K>(cw[j], sc[j], v);
-            rotate_unit<B, K>(v, lane, p.c_hi, p.c_lo);
-            const int64_t e0 = u * EPT;
-            if (e0 >= p.n) continue;
-            const bool full = e0 + EPT <= p.n;
+        for (int c0 = 0; c0 < DPL; c0 += CH) {
+            f32x2 v[CH / 2];
+#pragma unroll
+            for (int k = 0; k < CH / 8; ++k) {
+                const int kk = c0 / 8 + k;                             // code word index in the lane's 128
+                f32x2 g[4];
+                decode8(cw[kk], g);
+                const float sv = decode_scale(scb[(8 * kk) / EPB], p.fmt, G);
+                const f32x2 s2 = pk(sv, sv);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[4 * k + j] = K > 0 ? mul2_rounded(g[j], s2) : mul2(g[j], s2);
+            }
+            if constexpr (K > 0) {
+                fwht_inreg<CH, K>(v);
+                normalize<CH>(v, p.c_hi, p.c_lo);
+            }
+            const int64_t ec = e0 + c0;
+            const bool full = ec + CH <= p.n;
             if constexpr (F32OUT) {
-                float* dst = reinterpret_cast<float*>(p.y) + e0;
+                float* dst = reinterpret_cast<float*>(p.y) + ec;
                 if (full) {
 #pragma unroll
-                    for (int k = 0; k < EPT / 4; ++k)
-                        stg128(dst + 4 * k, __float_as_uint(v[4 * k]), __float_as_uint(v[4 * k + 1]),
-                               __float_as_uint(v[4 * k + 2]), __float_as_uint(v[4 * k + 3]));
+                    for (int k = 0; k < CH / 8; ++k) {
+                        float a[8];
+                        upk(v[4 * k], a[0], a[1]);
+                        upk(v[4 * k + 1], a[2], a[3]);
+                        upk(v[4 * k + 2], a[4], a[5]);
+                        upk(v[4 * k + 3], a[6], a[7]);
+                        stg256(dst + 8 * k, __float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                               __float_as_uint(a[3]), __float_as_uint(a[4]), __float_as_uint(a[5]),
+                               __float_as_uint(a[6]), __float_as_uint(a[7]));
+                    }
                 } else {
-                    for (int i = 0; i < EPT && e0 + i < p.n; ++i) dst[i] = v[i];
+#pragma unroll
+                    for (int k = 0; k < CH / 2; ++k) {
+                        float a, b;
+                        upk(v[k], a, b);
+                        if (ec + 2 * k < p.n) {
+                            dst[2 * k] = a;
+                            dst[2 * k + 1] = b;
+                        }
+                    }
                 }
             } else {
-                uint32_t o[EPT / 2];
+                uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.y) + ec);
 #pragma unroll
-                for (int k = 0; k < EPT / 2; ++k) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-                    o[k] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.y) + e0);
-                if (full) {
+                for (int k = 0; k < CH / 16; ++k) {
+                    uint32_t o[8];
 #pragma unroll
-                    for (int k = 0; k < EPT / 8; ++k) stg128(dst + 4 * k, o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-                } else {
-                    for (int k = 0; k < EPT / 2 && e0 + 2 * k < p.n; ++k) dst[k] = o[k];
+                    for (int j = 0; j < 8; ++j) {
+                        float a, b;
+                        upk(v[8 * k + j], a, b);
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+                        o[j] = *reinterpret_cast<uint32_t*>(&hb);
+                    }
+                    if (full) {
+                        stg256(dst + 8 * k, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (ec + 16 * k + 2 * j < p.n) dst[8 * k + j] = o[j];
+                    }
                 }
             }
         }
-    }
+    });
 }
 
-// ---------------------------------------------------------------- block MSE
+// ---------------------------------------------------------------- block MSE of given codes
 struct MseParams {
     const uint16_t* x;
     const uint8_t* codes;
@@ -463,149 +744,171 @@ __device__ __forceinline__ float tree_sum(const float* a)
     else return __fadd_rn(tree_sum<N / 2>(a), tree_sum<N / 2>(a + N / 2));
 }
 
-template <int LANES>
-__device__ __forceinline__ float group_sum(float s)
+// Codes and scale bytes of a unit (zeros past the end).
+template <int B, int K>
+__device__ __forceinline__ void load_unit_codes(const uint8_t* __restrict__ codes,
+                                                const uint8_t* __restrict__ scales, int64_t n, int64_t u,
+                                                uint32_t (&cw)[EPT / 8], uint32_t (&sb)[UnitShape<B, K>::NB])
 {
+    using S = UnitShape<B, K>;
+    const int64_t e0 = u * EPT;
+    if (e0 + EPT <= n) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4*>(codes + e0 / 2));
+        cw[0] = r.x;
+        cw[1] = r.y;
+        cw[2] = r.z;
+        cw[3] = r.w;
+    } else {
+        const int64_t nbytes = e0 < n ? (n - e0) / 2 : 0;
 #pragma unroll
-    for (int d = 1; d < LANES; d <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, d));
-    return s;
+        for (int k = 0; k < EPT / 8; ++k) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (4 * k + j < nbytes) word |= (uint32_t)codes[e0 / 2 + 4 * k + j] << (8 * j);
+            cw[k] = word;
+        }
+    }
+#pragma unroll
+    for (int bi = 0; bi < S::NB; ++bi) {
+        const int64_t e = e0 + (int64_t)bi * S::BE;
+        sb[bi] = e < n ? (uint32_t)__ldg(scales + e / B) : 0u;
+    }
 }
 
+// The codes may come from anywhere, so the block maximum's error is taken at
+// the first element of largest |y| (the oracle's reading), not from the
+// largest dequantized value.
 template <int B, int K>
 __global__ void __launch_bounds__(kThreads) block_mse_kernel(MseParams p)
 {
     using S = UnitShape<B, K>;
-    constexpr int EPT = S::EPT, U = S::UNITS, NB = S::kBlocksPerUnit, BE = S::kBlockElems;
-    constexpr int LPB = S::kLanesPerBlock;
+    constexpr int NB = S::NB, BE = S::BE, LPB = S::LPB;
+    extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
-    const int64_t n_units = (p.n + EPT - 1) / EPT;
-    const int64_t n_tiles = (n_units + 32 * U - 1) / (32 * U);
+    const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const XRing ring = warp_ring<XRing>(smem_ring);
     const float G = (p.fmt != kE8M0 && p.gsrc != nullptr) ? *p.gsrc : 1.0f;
 
     double acc_total = 0.0, acc_nonmax = 0.0, acc_max = 0.0, acc_zero = 0.0;
-    for (int64_t tile = warp; tile < n_tiles; tile += n_warps) {
-        uint32_t w[U][EPT / 2];
-        uint32_t cw[U][EPT / 8];
-        float sc[U][NB];
+    // codes and scales of the next tile are fetched one iteration ahead
+    uint32_t cw_next[EPT / 8], sb_next[NB];
+    if (warp < n_tiles) load_unit_codes<B, K>(p.codes, p.scales, p.n, warp * 32 + lane, cw_next, sb_next);
+    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
+                 [&](int64_t t, int s) {
+        const int64_t u = t * 32 + lane;
+        uint32_t cw[EPT / 8], sb[NB];
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            load_unit<EPT>(p.x, p.n, u, w[j]);
-            load_codes<EPT>(p.codes, p.n, u, cw[j]);
-            load_scales<B, K>(p.scales, p.fmt, G, p.n, u, sc[j]);
+        for (int k = 0; k < EPT / 8; ++k) cw[k] = cw_next[k];
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) sb[bi] = sb_next[bi];
+        if (t + n_warps < n_tiles) load_unit_codes<B, K>(p.codes, p.scales, p.n, (t + n_warps) * 32 + lane, cw_next, sb_next);
+        uint32_t w[EPT / 2];
+        ring.read(s, 0, w);
+        const int64_t e0 = u * EPT;
+        f32x2 yp[EPT / 2];
+        unpack_unit(w, yp);
+        rotate_unit<K>(yp, lane, p.c_hi, p.c_lo);
+        float m[NB];
+        block_max<B, K>(yp, m);
+        float y[EPT], v[EPT];
+#pragma unroll
+        for (int k = 0; k < EPT / 8; ++k) {
+            f32x2 g[4];
+            decode8(cw[k], g);
+            const int bi = (8 * k) / BE;
+            const float sv = e0 + (int64_t)bi * BE < p.n ? decode_scale(sb[bi], p.fmt, G) : 0.0f;
+            const f32x2 s2 = pk(sv, sv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                upk(mul2_rounded(g[j], s2), v[8 * k + 2 * j], v[8 * k + 2 * j + 1]);
+                upk(yp[4 * k + j], y[8 * k + 2 * j], y[8 * k + 2 * j + 1]);
+            }
         }
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t u = (tile * U + j) * 32 + lane;
-            const int64_t e0 = u * EPT;
-            float y[EPT], v[EPT];
-            unpack_unit<EPT>(w[j], y);
-            rotate_unit<B, K>(y, lane, p.c_hi, p.c_lo);
-            decode_unit<B, K>(cw[j], sc[j], v);
-            float m[NB];
-            block_max<B, K>(y, m);
+        for (int bi = 0; bi < NB; ++bi) {
+            float e2[BE];
+            float vmax = 0.0f;
+            int first = BE;                       // first element of largest |y| in this lane
 #pragma unroll
-            for (int bi = 0; bi < NB; ++bi) {
-                float e2[BE];
-                float vmax = 0.0f;
-                int first = BE;                       // first element of largest |y| in this lane
+            for (int i = BE - 1; i >= 0; --i) {
+                const float yi = y[bi * BE + i], vi = v[bi * BE + i];
+                const float d = __fsub_rn(yi, vi);
+                e2[i] = __fmul_rn(d, d);
+                vmax = fmaxf(vmax, fabsf(vi));
+                if (fabsf(yi) == m[bi]) first = i;
+            }
+            float emax = 0.0f;
 #pragma unroll
-                for (int i = BE - 1; i >= 0; --i) {
-                    const float yi = y[bi * BE + i], vi = v[bi * BE + i];
-                    const float d = __fsub_rn(yi, vi);
-                    e2[i] = __fmul_rn(d, d);
-                    vmax = fmaxf(vmax, fabsf(vi));
-                    if (fabsf(yi) == m[bi]) first = i;
-                }
-                float emax = 0.0f;
+            for (int i = 0; i < BE; ++i)
+                if (i == first) emax = e2[i];
+            bool owner = first < BE;
+            if constexpr (LPB > 1) {
+                // the block's maximum belongs to the lowest lane that holds it
+                const unsigned grp = (lane / LPB) * LPB;
+                const unsigned mask = ((LPB == 32) ? 0xffffffffu : ((1u << LPB) - 1u)) << grp;
+                const unsigned holders = __ballot_sync(0xffffffffu, owner) & mask;
+                owner = owner && (__ffs(holders) - 1 == lane);
+                vmax = group_max<LPB>(vmax);
+            }
+            const float sum = tree_sum<BE>(e2);
+            const float mx = owner ? emax : 0.0f;
+            float nm_arr[BE];
 #pragma unroll
-                for (int i = 0; i < BE; ++i) if (i == first) emax = e2[i];
-                bool owner = first < BE;
-                if constexpr (LPB > 1) {
-                    // the block's maximum belongs to the lowest lane that holds it
-                    const unsigned grp = (lane / LPB) * LPB;
-                    const unsigned mask = ((LPB == 32) ? 0xffffffffu : ((1u << LPB) - 1u)) << grp;
-                    const unsigned holders = __ballot_sync(0xffffffffu, owner) & mask;
-                    owner = owner && (__ffs(holders) - 1 == lane);
-                    vmax = group_max<LPB>(vmax);
-                }
-                const float sum = tree_sum<BE>(e2);
-                const float mx = owner ? emax : 0.0f;
-                // non-max part: every element except the owner's first maximum
-                float nm_arr[BE];
-#pragma unroll
-                for (int i = 0; i < BE; ++i) nm_arr[i] = (owner && i == first) ? 0.0f : e2[i];
-                float nonmax = tree_sum<BE>(nm_arr);
-                float bsum = sum, bmax = mx;
-                if constexpr (LPB > 1) {
-                    bsum = group_sum<LPB>(bsum);
-                    nonmax = group_sum<LPB>(nonmax);
-                    bmax = group_sum<LPB>(bmax);
-                }
-                const int64_t eb = e0 + (int64_t)bi * BE;
-                const bool leader = (LPB == 1) || ((lane % LPB) == 0);
-                if (leader && eb < p.n) {
-                    if (p.block_mse) p.block_mse[eb / B] = __fdiv_rn(bsum, (float)B);
-                    acc_total += (double)bsum;
-                    if (vmax == 0.0f) acc_zero += (double)bsum;
-                    else {
-                        acc_nonmax += (double)nonmax;
-                        acc_max += (double)bmax;
-                    }
+            for (int i = 0; i < BE; ++i) nm_arr[i] = (owner && i == first) ? 0.0f : e2[i];
+            float nonmax = tree_sum<BE>(nm_arr);
+            float bsum = sum, bmax = mx;
+            if constexpr (LPB > 1) {
+                bsum = group_sum<LPB>(bsum);
+                nonmax = group_sum<LPB>(nonmax);
+                bmax = group_sum<LPB>(bmax);
+            }
+            const int64_t eb = e0 + (int64_t)bi * BE;
+            const bool leader = (LPB == 1) || ((lane % LPB) == 0);
+            if (leader && eb < p.n) {
+                if (p.block_mse) p.block_mse[eb / B] = __fmul_rn(bsum, 1.0f / (float)B);
+                acc_total += (double)bsum;
+                if (vmax == 0.0f) acc_zero += (double)bsum;
+                else {
+                    acc_nonmax += (double)nonmax;
+                    acc_max += (double)bmax;
                 }
             }
         }
-    }
-    // deterministic block reduction: warp butterflies, then warps in order
-    __shared__ double red[kThreads / 32][4];
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) {
-        acc_total += __shfl_xor_sync(0xffffffffu, acc_total, d);
-        acc_nonmax += __shfl_xor_sync(0xffffffffu, acc_nonmax, d);
-        acc_max += __shfl_xor_sync(0xffffffffu, acc_max, d);
-        acc_zero += __shfl_xor_sync(0xffffffffu, acc_zero, d);
-    }
-    const int wid = threadIdx.x >> 5;
-    if (lane == 0) {
-        red[wid][0] = acc_total;
-        red[wid][1] = acc_nonmax;
-        red[wid][2] = acc_max;
-        red[wid][3] = acc_zero;
-    }
-    __syncthreads();
-    if (threadIdx.x < 4) {
-        double s = 0.0;
-        for (int k = 0; k < kThreads / 32; ++k) s += red[k][threadIdx.x];
-        p.partials[(int64_t)blockIdx.x * 4 + threadIdx.x] = s;
-    }
+    });
+    cta_partials(acc_total, acc_nonmax, acc_max, acc_zero, p.partials);
 }
 
 // terms[i] = (sum of partials[*][i]) / n, summed in a fixed order.
 static __global__ void __launch_bounds__(kThreads) mse_finalize_kernel(const double* partials, int nparts,
-                                                               int64_t n, double* terms)
+                                                                      int64_t n, double* terms)
 {
-    __shared__ double red[kThreads][4];
+    __shared__ double red[kWarps][4];
     double s[4] = {0.0, 0.0, 0.0, 0.0};
     for (int i = threadIdx.x; i < nparts; i += kThreads)
 #pragma unroll
         for (int k = 0; k < 4; ++k) s[k] += partials[(int64_t)i * 4 + k];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) red[threadIdx.x][k] = s[k];
-    __syncthreads();
-    for (int h = kThreads / 2; h >= 1; h >>= 1) {
-        if (threadIdx.x < h)
+    for (int d = 16; d >= 1; d >>= 1)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) red[threadIdx.x][k] += red[threadIdx.x + h][k];
-        __syncthreads();
+        for (int k = 0; k < 4; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], d);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) red[wid][k] = s[k];
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        double t = 0.0;
+        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
+        terms[threadIdx.x] = n > 0 ? t / (double)n : 0.0;
     }
-    if (threadIdx.x < 4) terms[threadIdx.x] = n > 0 ? red[0][threadIdx.x] / (double)n : 0.0;
 }
 
 // ---------------------------------------------------------------- element codecs
 static __global__ void __launch_bounds__(kThreads) e2m1_encode_kernel(const float* __restrict__ r, int64_t n,
-                                                              uint8_t* __restrict__ out)
+                                                                     uint8_t* __restrict__ out)
 {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; 8 * i < n; i += stride) {
@@ -622,17 +925,36 @@ static __global__ void __launch_bounds__(kThreads) e2m1_encode_kernel(const floa
     }
 }
 
+// Scale codes one value at a time through the quantizer's own block-scale
+// routines with 6 G = 1: UE formats give the code nearest to s, E8M0 the byte
+// of a block whose maximum is s.  UE4M3 goes through the paired routine the
+// quantizer uses for two blocks (values i and i + 1 form a pair).
 static __global__ void __launch_bounds__(kThreads) scale_encode_kernel(const float* __restrict__ s, int64_t n,
-                                                               int fmt, uint8_t* __restrict__ out)
+                                                                      int fmt, uint8_t* __restrict__ out)
 {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
-        const float v = s[i];
-        uint32_t c;
-        if (fmt == kE8M0) c = e8m0_from_amax(v);
-        else if (fmt == kUE4M3) c = ue4m3_encode(v);
-        else c = ue5m3_encode(v);
-        out[i] = (uint8_t)c;
+    ScaleConsts k1;
+    k1.G = 1.0f;
+    k1.denom = 1.0f;
+    k1.denom_ok = true;
+    k1.rd_lo = kBracketLo;
+    k1.rd_hi = kBracketHi;
+    for (int64_t i = 2 * ((int64_t)blockIdx.x * kThreads + threadIdx.x); i < n; i += 2 * stride) {
+        const float s0 = s[i], s1 = (i + 1 < n) ? s[i + 1] : 0.0f;
+        float S0, S1, a0, a1, b0, b1;
+        bool ok;
+        uint32_t c0, c1;
+        if (fmt == kE8M0) {
+            c0 = block_scale<kE8M0>(s0, k1, S0, a0, b0, ok);
+            c1 = block_scale<kE8M0>(s1, k1, S1, a1, b1, ok);
+        } else if (fmt == kUE4M3) {
+            block_scale_ue4m3_pair(s0, s1, k1, c0, c1, S0, S1, a0, a1, b0, b1);
+        } else {
+            c0 = block_scale<kUE5M3>(s0, k1, S0, a0, b0, ok);
+            c1 = block_scale<kUE5M3>(s1, k1, S1, a1, b1, ok);
+        }
+        out[i] = (uint8_t)c0;
+        if (i + 1 < n) out[i + 1] = (uint8_t)c1;
     }
 }
 

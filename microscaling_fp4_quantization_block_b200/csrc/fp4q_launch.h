@@ -11,20 +11,37 @@ struct AmaxParams;
 struct DequantParams;
 struct MseParams;
 
-// Grid size for a grid-stride kernel: enough CTAs for the work, at most the
-// number that fit on the device at once (occupancy x SM count).
-int resident_grid(const void* kernel, int64_t ctas_needed);
+// Opt a kernel in to `smem` bytes of dynamic shared memory (once per kernel
+// and device) and return how many of its CTAs fit on the device at once.
+int resident_ctas(const void* kernel, int smem);
+
+// Grid for a grid-stride kernel: min(ctas_needed, resident CTAs), at least 1.
+int grid_for(const void* kernel, int smem, int64_t ctas_needed);
+
+// CTAs a ring kernel needs for n elements (one 32-unit tile per warp).
+int64_t ring_ctas_needed(int64_t n, int ept);
 
 // Each returns cudaSuccess or the launch error; an unsupported (fmt, B, K)
 // combination returns cudaErrorInvalidValue before launching anything.
-cudaError_t launch_quantize(int fmt, int B, int K, const QuantParams& p, cudaStream_t s);
+// launch_quantize with mse = true writes per-CTA partials (grid <= max_grid).
+cudaError_t launch_quantize(int fmt, int B, int K, bool mse, const QuantParams& p, int* grid_out,
+                            cudaStream_t s);
+cudaError_t launch_quantize_e8m0(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
+cudaError_t launch_quantize_ue4m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
+cudaError_t launch_quantize_ue5m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s);
 cudaError_t launch_dequantize(int B, int K, bool f32out, const DequantParams& p, cudaStream_t s);
-cudaError_t launch_block_mse(int B, int K, const MseParams& p, int grid, cudaStream_t s);
-int mse_grid(int B, int K, int64_t n);
+cudaError_t launch_block_mse(int B, int K, const MseParams& p, int* grid_out, cudaStream_t s);
 
-// Elements one warp-tile covers (32 lanes x units in flight x elements per unit).
-constexpr int64_t kTileElems = 2048;
-constexpr int kMaxMseCtas = 4096;
+// Upper bound on the CTAs of any kernel that writes per-CTA partials, and the
+// number of partial slots (4 doubles each) a workspace must hold for n elements.
+constexpr int kMaxPartialCtas = 4096;
+constexpr int64_t kElemsPerPartial = 4096;
+inline int64_t partial_slots(int64_t n)
+{
+    int64_t s = (n + kElemsPerPartial - 1) / kElemsPerPartial;
+    if (s < 1) s = 1;
+    return s < kMaxPartialCtas ? s : kMaxPartialCtas;
+}
 
 }  // namespace fp4q

@@ -1,0 +1,56 @@
+// fp4q_quantize_impl.cuh -- template dispatch of the quantize kernel for one
+// scale format (each format is its own translation unit, built in parallel).
+#pragma once
+
+#include "fp4q_kernels.cuh"
+#include "fp4q_launch.h"
+
+namespace fp4q {
+namespace detail {
+
+template <int FMT, int B, int K, bool MSE>
+cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
+{
+    auto kern = quantize_kernel<FMT, B, K, MSE>;
+    int64_t need = ring_ctas_needed(p.n, EPT);
+    if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
+    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
+    if (grid_out) *grid_out = grid;
+    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int FMT, int B, int K>
+cudaError_t by_mse(bool mse, const QuantParams& p, int* g, cudaStream_t s)
+{
+    return mse ? run_quantize<FMT, B, K, true>(p, g, s) : run_quantize<FMT, B, K, false>(p, g, s);
+}
+
+template <int FMT, int B>
+cudaError_t by_rot(int K, bool mse, const QuantParams& p, int* g, cudaStream_t s)
+{
+    switch (K) {
+    case 0: return by_mse<FMT, B, 0>(mse, p, g, s);
+    case 16: return by_mse<FMT, B, 16>(mse, p, g, s);
+    case 32: return by_mse<FMT, B, 32>(mse, p, g, s);
+    case 128: return by_mse<FMT, B, 128>(mse, p, g, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT>
+cudaError_t by_block(int B, int K, bool mse, const QuantParams& p, int* g, cudaStream_t s)
+{
+    switch (B) {
+    case 8: return by_rot<FMT, 8>(K, mse, p, g, s);
+    case 16: return by_rot<FMT, 16>(K, mse, p, g, s);
+    case 32: return by_rot<FMT, 32>(K, mse, p, g, s);
+    case 64: return by_rot<FMT, 64>(K, mse, p, g, s);
+    case 128: return by_rot<FMT, 128>(K, mse, p, g, s);
+    case 256: return by_rot<FMT, 256>(K, mse, p, g, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace detail
+}  // namespace fp4q

@@ -47,9 +47,10 @@ def gpu_run(fq, x: torch.Tensor, fmt: int, block: int, rot: int, gmode: int, gva
     if want_mse:
         out["bm"], out["terms"] = fq.fp4q_block_mse(xd, codes, scales, gptr, fmt, block, rot)
     torch.cuda.synchronize()
-    res = {k: v.cpu().numpy() for k, v in out.items()}
-    if "deqbf" in res:
-        res["deqbf"] = out["deqbf"].cpu().view(torch.int16).numpy().view(np.uint16)
+    res = {}
+    for k, v in out.items():
+        v = v.cpu()
+        res[k] = v.view(torch.int16).numpy().view(np.uint16) if v.dtype == torch.bfloat16 else v.numpy()
     res["codes"] = codes.cpu().numpy()
     res["scales"] = scales.cpu().numpy()
     res["G"] = float(gs.item()) if gs is not None else 1.0

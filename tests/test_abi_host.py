@@ -102,6 +102,10 @@ def test_dequantize_and_mse_reject_bad_arguments(fp4q):
     assert L.fp4q_e2m1_encode_f32(A32, 7, A32, None) == -2                            # odd count
     assert L.fp4q_scale_encode_f32(A32, 8, 9, A32, None) == -4
     assert L.fp4q_e2m1_encode_f32(None, 0, None, None) == 0
+    assert L.fp4q_quantize_mse(A32, 4, 64, 1, 16, 0, 0, A32, A32, None, None, None, A32, ws, None) == -1
+    assert L.fp4q_quantize_mse(A32, 4, 64, 1, 16, 0, 0, A32, A32, None, None, A32, A32, ws - 8, None) == -6
+    assert L.fp4q_quantize_mse(A32, 4, 64, 0, 32, 0, 1, A32, A32, A32, None, A32, A32, ws, None) == -4
+    assert L.fp4q_quantize_mse(A32, 4, 64, 1, 16, 0, 0, A32, A32, None, A32 + 8, A32, A32, ws, None) == -3
     assert L.fp4q_global_scale(None, A32, None) == -1
     assert L.fp4q_global_scale(A32 + 2, A32, None) == -3
 

@@ -57,9 +57,12 @@ def _check_sampled(fq, xd, codes, scales, gs, bm, fmt, block, rot, gmode, G_orac
 
 
 def _terms_consistent(bm, terms):
+    """The GPU sums each block's squared errors in fp32 (all of them, and
+    separately the non-max ones), so the parts add up to the total to fp32
+    rounding; the total is the mean of the per-block MSE to the same bound."""
     t = terms.cpu().numpy()
-    assert t[0] == pytest.approx(t[1] + t[2] + t[3], rel=1e-12, abs=1e-300)
-    assert t[0] == pytest.approx(bm.double().mean().item(), rel=1e-9)
+    assert t[0] == pytest.approx(t[1] + t[2] + t[3], rel=2e-6, abs=1e-300)
+    assert t[0] == pytest.approx(bm.double().mean().item(), rel=2e-6)
 
 
 def test_nvfp4_qwen25_7b_mlp_full(fq):
@@ -105,8 +108,12 @@ def test_qwen25_14b_weight_pass(fq):
     """48 layers x {q, k, v, o, gate, up, down}, sigma_l = 0.02 * U(0.5, 1.5);
     MXFP4 and NVFP4 (per-tensor scale), without and with a 32-wide rotation.
     Sampled rows of every layer's first tensor (and of every tensor of every
-    sixth layer) against the oracle; every layer's unrotated MSE split against
-    the Gaussian model (per-tensor G for NVFP4)."""
+    sixth layer) against the oracle; the whole k projection of every fourth
+    layer against the oracle's MSE terms; every layer's split against the
+    Gaussian model as a sanity bound (bf16 rounding of the inputs moves block
+    maxima onto the power-of-two and scale-code boundaries where the
+    max-element error jumps, so the continuous model is only good to ~1-2%
+    for the max term at this size)."""
     sigmas = workloads.layer_sigmas(workloads.QWEN25_14B_LAYERS, 0.02, 0.5, seed=14)
     variants = [(E8, 32, 0, NONE), (U4, 16, 0, COMP), (E8, 32, 32, NONE), (U4, 16, 32, COMP)]
     for layer, sigma in enumerate(sigmas):
@@ -118,20 +125,28 @@ def test_qwen25_14b_weight_pass(fq):
             x = workloads.gaussian_bf16(t.rows, t.cols, sigma, seed=100000 + 16 * layer + ti, device="cuda")
             layer_n += n
             check = (layer % 6 == 0) or ti == 0
+            whole = (layer % 4 == 0) and t.name == "k"
+            xh = bf16_bits(x) if whole else None
             for v in variants:
                 fmt, block, rot, gmode = v
                 codes, scales, gs, bm, terms = _run_full(fq, x, fmt, block, rot, gmode)
-                got[v] += terms.cpu().numpy() * n
+                tt = terms.cpu().numpy()
+                got[v] += tt * n
                 G = float(gs.item()) if gs is not None else 1.0
                 if v in want:
                     want[v] += np.array(theory.three_terms(fmt, block, sigma, G)) * n
                 if check:
                     _check_sampled(fq, x, codes, scales, gs, bm, fmt, block, rot, gmode, G,
                                    _sample_rows(t.rows, 2, layer * 7 + ti))
+                if whole and (rot == 0 or layer % 12 == 0):
+                    _, o_terms = oracle.block_mse(xh, codes.cpu().numpy(), scales.cpu().numpy(), G, fmt,
+                                                  block, rot)
+                    for i in range(4):
+                        assert abs(tt[i] - o_terms[i]) <= (2e-6 if rot == 0 else 1e-5) * o_terms[0]
         for v in variants:
             tl = got[v] / layer_n
-            assert tl[0] == pytest.approx(tl[1] + tl[2] + tl[3], rel=1e-12)
+            assert tl[0] == pytest.approx(tl[1] + tl[2] + tl[3], rel=2e-6)
             if v in want:
                 th = want[v] / layer_n
-                assert tl[1] == pytest.approx(th[0], rel=2e-3), (layer, v, tl, th)
-                assert tl[2] == pytest.approx(th[1], rel=6e-3), (layer, v, tl, th)
+                assert tl[1] == pytest.approx(th[0], rel=1e-2), (layer, v, tl, th)
+                assert tl[2] == pytest.approx(th[1], rel=4e-2), (layer, v, tl, th)
