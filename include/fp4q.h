@@ -176,6 +176,34 @@ FP4Q_API int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fm
 FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block);
 
 /*
+ * fp4q_block_mse_noalloc -- fp4q_block_mse without a workspace argument, for
+ * callers that cannot allocate device memory (code running where no
+ * allocation may happen, or a host that owns no device allocator and
+ * would have nowhere to get the workspace from).  The pages have no
+ * counterpart: this is an interface convenience, not a step of the method.
+ *
+ * Same arguments, results and errors as fp4q_block_mse; the per-CTA partials
+ * live in a fixed static device buffer of libfp4q.so instead of a caller
+ * workspace.  The library allocates nothing (no cudaMalloc, no allocating
+ * library routine).
+ *  - Limit: the buffer holds 4096 partial slots (128 KiB).  The MSE kernel
+ *    never uses more, whatever the tensor size; a launch that would need more
+ *    returns FP4Q_ERR_WORKSPACE before anything is enqueued.
+ *  - Setup: the first call on each device (with that device current) looks
+ *    up the buffer's device address with cudaGetSymbolAddress and caches it.
+ *    Make that first call before any stream capture begins on the device.
+ *  - Nothing needs to start at zero: every launched CTA overwrites its own
+ *    slot before the final reduction reads it.
+ *  - One buffer per device: two calls in flight at the same time on one
+ *    device (on different streams, or from different host threads without
+ *    ordering) race on it and give wrong terms.  Calls ordered on one stream
+ *    are safe.
+ */
+FP4Q_API int fp4q_block_mse_noalloc(const void* x, const uint8_t* codes, const uint8_t* scales,
+                                    const float* gscale, int64_t rows, int64_t cols, int fmt, int block,
+                                    int rot, float* block_mse, double* terms, void* stream);
+
+/*
  * Element and scale codecs on their own, one value at a time ("Bridging the
  * Gap", s1; "Finer is better?", Theoretical framework and Contributions).
  * fp4q_e2m1_encode_f32: nibble of the E2M1 value nearest to r[i] (the rule of

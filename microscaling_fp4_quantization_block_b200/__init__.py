@@ -48,6 +48,7 @@ def _load() -> ctypes.CDLL:
         "fp4q_dequantize": (I, [P, P, P, I64, I64, I, I, I, I, P, P]),
         "fp4q_block_mse": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P, SZ, P]),
         "fp4q_block_mse_workspace_size": (SZ, [I64, I64, I]),
+        "fp4q_block_mse_noalloc": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P]),
         "fp4q_quantize_mse": (I, [P, I64, I64, I, I, I, I, P, P, P, P, P, P, SZ, P]),
         "fp4q_e2m1_encode_f32": (I, [P, I64, P, P]),
         "fp4q_scale_encode_f32": (I, [P, I64, I, P, P]),
@@ -199,6 +200,28 @@ def fp4q_block_mse(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
                              block, rot, _ptr(block_mse), _ptr(terms), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "fp4q_block_mse")
+    return block_mse, terms
+
+
+def fp4q_block_mse_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                           gscale: Optional[torch.Tensor], fmt, block: int, rot: int = 0,
+                           block_mse: Optional[torch.Tensor] = None, terms: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[Optional[torch.Tensor], torch.Tensor]:
+    """fp4q_block_mse with the library's fixed device scratch instead of a
+    workspace, for callers that cannot allocate device memory: with
+    ``block_mse`` and ``terms`` passed in, this function allocates nothing
+    (block_mse may be None to skip the per-block output).  Calls in flight at
+    the same time on one device race on the shared scratch; calls ordered on
+    one stream do not."""
+    _need_cuda(x, codes, scales, gscale)
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous (no copy is made here)")
+    rows, cols = x.shape
+    if terms is None:
+        terms = torch.empty((4,), dtype=torch.float64, device=x.device)
+    st = lib().fp4q_block_mse_noalloc(_ptr(x), _ptr(codes), _ptr(scales), _ptr(gscale), rows, cols, _fmt(fmt),
+                                      block, rot, _ptr(block_mse), _ptr(terms), _stream(stream))
+    _check(st, "fp4q_block_mse_noalloc")
     return block_mse, terms
 
 

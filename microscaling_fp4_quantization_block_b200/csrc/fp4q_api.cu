@@ -2,6 +2,7 @@
 // launches.  Nothing here allocates device memory or synchronizes.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/fp4q.h"
 #include "fp4q_kernels.cuh"
@@ -59,6 +60,34 @@ cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStre
     ap.amax_bits = reinterpret_cast<unsigned int*>(dst);
     rotation_constants(rot, &ap.c_hi, &ap.c_lo);
     return launch_amax(rot, ap, s);
+}
+
+// ---- fixed scratch of fp4q_block_mse_noalloc
+// Per-CTA MSE partials for callers that cannot allocate a workspace: one
+// static device buffer per device, 4096 slots of 4 doubles (128 KiB), which is
+// the most partial slots any launch uses (the MSE kernel caps its grid there).
+constexpr int kNoAllocSlots = kMaxPartialCtas;
+static __device__ __align__(256) double g_noalloc_partials[kNoAllocSlots * 4];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+double* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_partials on the current device, looked up with
+// cudaGetSymbolAddress the first time each device is seen.
+int noalloc_partials_for_current_device(double** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || !p) return FP4Q_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<double*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return FP4Q_OK;
 }
 
 }  // namespace
@@ -268,6 +297,44 @@ int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, vo
     if (!aligned(s, 4) || !aligned(codes, 4)) return FP4Q_ERR_ALIGN;
     int grid = grid_for((const void*)scale_encode_kernel, 0, (n + kThreads - 1) / kThreads);
     scale_encode_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(s, n, fmt, codes);
+    return cuda_status(cudaGetLastError());
+}
+
+int fp4q_block_mse_noalloc(const void* x, const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                           int64_t rows, int64_t cols, int fmt, int block, int rot, float* block_mse,
+                           double* terms, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (!terms) return FP4Q_ERR_NULL;
+    if (n > 0 && (!x || !codes || !scales)) return FP4Q_ERR_NULL;
+    if (!aligned(terms, 8)) return FP4Q_ERR_ALIGN;
+    if (gscale && !aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)))
+        return FP4Q_ERR_ALIGN;
+    if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
+    if (partial_slots(n) > kNoAllocSlots) return FP4Q_ERR_WORKSPACE;
+    double* partials = nullptr;
+    st = noalloc_partials_for_current_device(&partials);
+    if (st) return st;
+    cudaStream_t s = as_stream(stream);
+    int grid = 0;
+    if (n > 0) {
+        MseParams p{};
+        p.x = static_cast<const uint16_t*>(x);
+        p.codes = codes;
+        p.scales = scales;
+        p.gsrc = gscale;
+        p.n = n;
+        p.fmt = fmt;
+        p.block_mse = block_mse;
+        p.partials = partials;
+        rotation_constants(rot, &p.c_hi, &p.c_lo);
+        // the launch uses at most partial_slots(n) CTAs, checked above to fit the scratch
+        if (launch_block_mse(block, rot, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
     return cuda_status(cudaGetLastError());
 }
 
