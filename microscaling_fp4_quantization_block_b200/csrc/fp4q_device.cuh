@@ -28,6 +28,33 @@ __device__ __forceinline__ uint32_t as_u32(float f) { return __float_as_uint(f);
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return as_f32(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return as_f32(w & 0xffff0000u); }
 
+// The high half widened by a mixed-precision add of -0 (bf16 + fp32 -> fp32,
+// exact): it issues on the floating-point pipe instead of the integer/logic
+// pipe that the mask above uses, which the rest of the quantizer keeps busy.
+__device__ __forceinline__ float bf16_hi_fp(uint32_t w)
+{
+    float r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %2;\n\t}"
+        : "=f"(r)
+        : "r"(w), "f"(-0.0f));
+    return r;
+}
+
+// Per half, max(|a|, |b|) of two bf16x2 words; the result's sign bits are
+// meaningless (xor of the inputs' signs) and are dropped by bf16x2_absmax_f32.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Larger magnitude of the two halves of a bf16x2 word, as fp32 (exact).
+__device__ __forceinline__ float bf16x2_absmax_f32(uint32_t m)
+{
+    return fmaxf(as_f32((m << 16) & 0x7fffffffu), as_f32(m & 0x7fff0000u));
+}
+
 // ---------------------------------------------------------------- vector memory
 struct alignas(32) U32x8 { uint32_t v[8]; };
 
@@ -81,15 +108,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t smem_addr)
     return r;
 }
 
-// Approximate reciprocal (at most 1 ulp from 1/s for normal s with a normal
-// reciprocal); only used where a bound, not the rounded value, matters.
-__device__ __forceinline__ float rcp_approx(float s)
-{
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
-    return r;
-}
-
 // ---------------------------------------------------------------- E2M1
 // Four pairs -> one 32-bit word of nibbles: byte k = code(v[2k]) | code(v[2k+1]) << 4.
 // cvt.rn.satfinite.e2m1x2.f32 rounds to nearest even onto the E2M1 grid,
@@ -122,6 +140,19 @@ __device__ __forceinline__ void e2m1_unpack2(uint32_t byte, float& lo, float& hi
     __half2 hh = *reinterpret_cast<__half2*>(&h2);
     lo = __low2float(hh);
     hi = __high2float(hh);
+}
+
+// Magnitude of the E2M1 grid value that q rounds to (E2M1 code, then its
+// value, through the two hardware conversions).
+__device__ __forceinline__ float e2m1_grid_value(float q)
+{
+    uint32_t h2;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %1, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
+        : "=r"(h2)
+        : "f"(q));
+    return fabsf(__half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu))));
 }
 
 // ---------------------------------------------------------------- E8M0
@@ -194,13 +225,6 @@ __device__ __forceinline__ void ue4m3_decode2_hw(uint32_t c2, float& lo, float& 
     hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
 }
 
-// Exact UE4M3 code of fp32(m / d): the fallback of the bracketed scale rule,
-// kept out of line so the common path carries none of its instructions.
-static __device__ __noinline__ uint32_t ue4m3_code_of_quotient(float m, float d)
-{
-    return ue4m3_encode(__fdiv_rn(m, d));
-}
-
 // ---------------------------------------------------------------- UE5M3
 // Nearest UE5M3 code to s >= 0 by integer rounding of the fp32 pattern: keep 3
 // mantissa bits with round-to-nearest-even (a carry moves into the exponent);
@@ -267,6 +291,14 @@ __device__ __forceinline__ f32x2 mul2_rounded(f32x2 a, f32x2 b)
     return pk(__fmul_rn(a0, b0), __fmul_rn(a1, b1));
 }
 
+// a * b + c with one rounding toward minus infinity, on both lanes.
+__device__ __forceinline__ f32x2 fma2_rm(f32x2 a, f32x2 b, f32x2 c)
+{
+    f32x2 r;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
 {
     f32x2 r;
@@ -300,31 +332,38 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return r;
 }
 
-// ---------------------------------------------------------------- block scale
-// Quotients that decide a code are bracketed instead of divided.  With an
-// approximate reciprocal R of a divisor d (at most 1 ulp off) and
-// R_lo = fp32(R (1 - 2^-19)), R_hi = fp32(R (1 + 2^-19)), the correctly rounded
-// quotient q* = fp32(a / d) lies strictly between fp32(a R_lo) and fp32(a R_hi)
-// for every fp32 a (the worst-case rounding errors add up to 6 units of 2^-24
-// against a bracket half-width of 32 units).  Rounding to E2M1 or to UE4M3 is
-// monotone in |q| and keeps the sign, so when both ends round to the same code
-// that code is the code of q*; otherwise the code is recomputed from the
-// correctly rounded division.  d and 1/d must both be normal floats.
-constexpr float kBracketLo = 0.99999809265136719f;   // 1 - 2^-19, exact in fp32
-constexpr float kBracketHi = 1.00000190734863281f;                           // 1 + 2^-19, exact in fp32
-
-__device__ __forceinline__ bool divisor_safe(float d)
+// ---------------------------------------------------------------- correctly rounded quotients
+// A quotient a / b that decides a code (element y / S, scale m / fp32(6G)) is
+// computed exactly, without a divide, from the correctly rounded reciprocal
+// R = fp32(1/b) (one per scale, not per element) by the remainder correction
+// of Markstein's division theorem:
+//   q0 = fp32(a R),   r = a - q0 b (exact; one fused multiply-add),
+//   q  = fp32(q0 + r R)  =  fp32(a / b).
+// The remainder is rounded toward minus infinity only so that an exact zero
+// remainder is -0: then a = -0 gives q = -0 and keeps its sign, as a true
+// division does; a non-zero remainder is exact and unaffected.  The identity is
+// checked on the GPU exhaustively for every bf16 significand a against every
+// fp32 significand b, both signs (the values the unrotated path divides), and
+// on random fp32 pairs; it needs b, 1/b and the quotient normal, so callers
+// keep b within [2^-100, 2^100] and |a / b| below 2^60 and divide otherwise.
+__device__ __forceinline__ f32x2 div2_cr(f32x2 a, f32x2 R, f32x2 neg_b)
 {
-    const uint32_t e = as_u32(d) >> 23;            // d > 0: biased exponent
-    return e >= 1u && e <= 252u;                   // d and 1/d normal
+    const f32x2 q0 = mul2(a, R);
+    const f32x2 r = fma2_rm(q0, neg_b, a);
+    return fma2(r, R, q0);
 }
 
-// Per-tensor constants of the UE scale rule.
+constexpr float kDivLo = 0x1p-100f;     // range of divisors the remainder correction serves
+constexpr float kDivHi = 0x1p100f;
+constexpr float kQuotMax = 0x1p60f;
+
+// Per-tensor constants of the UE scale rule: G, the divisor fp32(6G) of the
+// block maxima and its correctly rounded reciprocal.
 struct ScaleConsts {
-    float G;                 // per-tensor scale
+    float G;
     float denom;             // fp32(6 G)
-    float rd_lo, rd_hi;      // bracket of 1/denom
-    bool denom_ok;
+    float rdenom;            // fp32(1 / denom), when denom_ok
+    bool denom_ok;           // denom within [2^-100, 2^100]
 };
 
 __device__ __forceinline__ ScaleConsts scale_consts(float G)
@@ -332,79 +371,9 @@ __device__ __forceinline__ ScaleConsts scale_consts(float G)
     ScaleConsts c;
     c.G = G;
     c.denom = __fmul_rn(6.0f, G);
-    c.denom_ok = divisor_safe(c.denom);
-    const float r = rcp_approx(c.denom);
-    c.rd_lo = __fmul_rn(r, kBracketLo);
-    c.rd_hi = __fmul_rn(r, kBracketHi);
+    c.denom_ok = c.denom >= kDivLo && c.denom <= kDivHi;
+    c.rdenom = c.denom_ok ? __frcp_rn(c.denom) : 0.0f;
     return c;
-}
-
-// UE4M3 scales of two blocks at once (block maxima m0, m1): codes, block
-// scales S = fp32(decode(code) G) and the brackets [r_lo, r_hi] of 1/S (both 0
-// for a zero block).  Returns false when some 1/S cannot be bracketed (S or
-// 1/S not a normal float), i.e. when elements must be divided.
-__device__ __forceinline__ bool block_scale_ue4m3_pair(float m0, float m1, const ScaleConsts& k, uint32_t& c0,
-                                                       uint32_t& c1, float& S0, float& S1, float& rlo0, float& rlo1,
-                                                       float& rhi0, float& rhi1)
-{
-    const f32x2 mm = pk(m0, m1);
-    float l0, l1, h0, h1;
-    upk(mul2(mm, pk(k.rd_lo, k.rd_lo)), l0, l1);
-    upk(mul2(mm, pk(k.rd_hi, k.rd_hi)), h0, h1);
-    uint32_t codes = ue4m3_encode2(l0, l1);                    // low byte: block 0
-    if (codes != ue4m3_encode2(h0, h1) || !k.denom_ok)         // rare: a quotient at a rounding tie
-        codes = ue4m3_code_of_quotient(m0, k.denom) | (ue4m3_code_of_quotient(m1, k.denom) << 8);
-    c0 = codes & 0xffu;
-    c1 = codes >> 8;
-    float d0, d1;
-    ue4m3_decode2_hw(codes, d0, d1);
-    upk(mul2(pk(d0, d1), pk(k.G, k.G)), S0, S1);
-    const f32x2 r = pk(rcp_approx(S0), rcp_approx(S1));
-    float a0, a1, b0, b1;
-    upk(mul2(r, pk(kBracketLo, kBracketLo)), a0, a1);
-    upk(mul2(r, pk(kBracketHi, kBracketHi)), b0, b1);
-    rlo0 = S0 == 0.0f ? 0.0f : a0;                             // zero-rounded block
-    rhi0 = S0 == 0.0f ? 0.0f : b0;
-    rlo1 = S1 == 0.0f ? 0.0f : a1;
-    rhi1 = S1 == 0.0f ? 0.0f : b1;
-    return (S0 == 0.0f || divisor_safe(S0)) && (S1 == 0.0f || divisor_safe(S1));
-}
-
-// Scale byte of a block with absolute maximum m ("max" rule), the block's
-// dequantization scale S and the bracket [r_lo, r_hi] of 1/S (0 for a zero
-// block; `exact` false when 1/S cannot be bracketed and elements must divide).
-//   E8M0:  S = 2^(floor(log2 m) - 2), r_lo = r_hi = 1/S exactly.
-//   UE4M3: the paired routine above on (m, m).
-//   UE5M3: s = code nearest fp32(m / denom) (exact division), S = fp32(decode(s) G).
-template <int FMT>
-__device__ __forceinline__ uint32_t block_scale(float m, const ScaleConsts& k, float& S, float& r_lo,
-                                                float& r_hi, bool& exact)
-{
-    uint32_t c;
-    if constexpr (FMT == kE8M0) {
-        c = e8m0_from_amax(m);
-        S = e8m0_decode(c);
-        r_lo = r_hi = e8m0_inverse(c);
-        exact = true;
-        return c;
-    } else if constexpr (FMT == kUE4M3) {
-        uint32_t c1;
-        float S1, a1, b1;
-        exact = block_scale_ue4m3_pair(m, m, k, c, c1, S, S1, r_lo, a1, r_hi, b1);
-        return c;
-    } else {
-        c = ue5m3_encode(__fdiv_rn(m, k.denom));
-        S = __fmul_rn(ue5m3_decode(c), k.G);
-        if (S == 0.0f) {
-            r_lo = r_hi = 0.0f;
-            exact = true;
-        } else {
-            const float r = rcp_approx(S);
-            upk(mul2(pk(r, r), pk(kBracketLo, kBracketHi)), r_lo, r_hi);
-            exact = divisor_safe(S);
-        }
-        return c;
-    }
 }
 
 // ---------------------------------------------------------------- Hadamard

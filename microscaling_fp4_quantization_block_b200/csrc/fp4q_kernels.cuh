@@ -21,7 +21,12 @@
 //
 // Arithmetic.  Element values live as fp32 pairs (f32x2) so that products,
 // sums and butterflies issue as packed two-wide instructions; the scales of
-// two blocks are computed together the same way.
+// two blocks are computed together the same way.  The quantizer keeps its
+// work on the floating-point (FMA) pipe where it can: on sm_100 the integer /
+// logic pipe that runs converts, permutes, min/max and compares issues at
+// half the rate, so codes come from exactly computed quotients (div2_cr) and
+// one convert per pair, bf16 is widened by a mixed-precision add, and unrotated
+// block maxima use packed bf16 magnitude maxima.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -164,11 +169,12 @@ __device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __res
 
 using XRing = Ring<2 * EPT, 1>;                                  // one bf16 unit per lane per tile
 
-// bf16 words -> fp32 pairs (exact widening).
+// bf16 words -> fp32 pairs (exact widening; shift for the low half, a
+// mixed-precision add for the high half, both on the floating-point pipe).
 __device__ __forceinline__ void unpack_unit(const uint32_t (&w)[EPT / 2], f32x2 (&p)[EPT / 2])
 {
 #pragma unroll
-    for (int k = 0; k < EPT / 2; ++k) p[k] = pk(bf16_lo(w[k]), bf16_hi(w[k]));
+    for (int k = 0; k < EPT / 2; ++k) p[k] = pk(bf16_lo(w[k]), bf16_hi_fp(w[k]));
 }
 
 // Optional rotation of a unit held in registers: runs of K elements, the part
@@ -203,6 +209,23 @@ __device__ __forceinline__ void block_max(const f32x2 (&p)[EPT / 2], float (&m)[
     using S = UnitShape<B, K>;
 #pragma unroll
     for (int bi = 0; bi < S::NB; ++bi) m[bi] = pairs_absmax<S::BE>(p + bi * S::BE / 2);
+    if constexpr (S::LPB > 1) m[0] = group_max<S::LPB>(m[0]);
+}
+
+// The same maxima straight from the bf16 words of an unrotated unit: packed
+// two-wide magnitude maxima, then the larger half (exact).
+template <int B>
+__device__ __forceinline__ void block_max_words(const uint32_t (&w)[EPT / 2], float (&m)[UnitShape<B, 0>::NB])
+{
+    using S = UnitShape<B, 0>;
+    constexpr int WPB = S::BE / 2;                                  // words of a block in this unit
+#pragma unroll
+    for (int bi = 0; bi < S::NB; ++bi) {
+        uint32_t a = w[bi * WPB];
+#pragma unroll
+        for (int k = 1; k < WPB; ++k) a = bf16x2_absmax(a, w[bi * WPB + k]);
+        m[bi] = bf16x2_absmax_f32(a);
+    }
     if constexpr (S::LPB > 1) m[0] = group_max<S::LPB>(m[0]);
 }
 
@@ -263,8 +286,9 @@ __device__ __forceinline__ uint32_t pack_pairs(f32x2 p0, f32x2 p1, f32x2 p2, f32
     return e2m1_pack8(a0, b0, a1, b1, a2, b2, a3, b3);
 }
 
-// Codes of 4 pairs with correctly rounded quotients v / s (s != 0): the rare
-// fallback of the bracketed element rounding, kept out of line.
+// Codes of 4 pairs with correctly rounded quotients v / s (s != 0) by
+// division: the fallback for scales outside the range the remainder
+// correction serves (extreme per-tensor scales), kept out of line.
 static __device__ __noinline__ uint32_t pack_pairs_div(f32x2 p0, f32x2 p1, f32x2 p2, f32x2 p3, float s)
 {
     float a[8];
@@ -277,72 +301,94 @@ static __device__ __noinline__ uint32_t pack_pairs_div(f32x2 p0, f32x2 p1, f32x2
     return e2m1_pack8(a[0], a[1], a[2], a[3], a[4], a[5], a[6], a[7]);
 }
 
-// Exact codes of 8 elements whose bracketed codes a (low end) and b (high end)
-// differ in some nibble: a quotient that sits at, or within 2^-18 of, an E2M1
-// rounding threshold t.  For such an element |y| and t S agree to ~8 bits, so
-// r = |y| - t S is exact through one fused multiply-add, and the correctly
-// rounded quotient fp32(|y| / S) equals t exactly when -h_lo S <= r <= h_hi S,
-// h being half the fp32 spacing below / above t (powers of two, so h S is
-// exact).  Then: r above the band -> the upper code, below -> the lower code,
-// inside -> the even one of the two (round half to even).  Elements whose two
-// codes agree keep them.  Kept out of line: it runs for ~0.1% of the words of
-// bf16 data whose per-tensor scale makes quotients land on thresholds.
-static __device__ __noinline__ uint32_t resolve_ties(uint32_t a, uint32_t b, f32x2 p0, f32x2 p1, f32x2 p2,
-                                                     f32x2 p3, float S)
+// Per-tensor table of the UE block scales, tab[c] = {S, R}: S = fp32(decode(c)
+// G) and R = fp32(1/S) correctly rounded; R = 0 for S = 0 (a zero-rounded
+// block), R = +inf for S outside [2^-100, 2^100] or a NaN code, which makes
+// the block divide instead (see unit_scales).
+template <int FMT>
+__device__ __forceinline__ void fill_scale_table(float2* tab, float G)
 {
-    float y[8];
-    upk(p0, y[0], y[1]);
-    upk(p1, y[2], y[3]);
-    upk(p2, y[4], y[5]);
-    upk(p3, y[6], y[7]);
-    f32x2 gl[4], gh[4];
-    decode8(a, gl);
-    decode8(b, gh);
-    uint32_t out = a;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t ca = (a >> (4 * j)) & 0xfu, cb = (b >> (4 * j)) & 0xfu;
-        if (ca == cb) continue;
-        float la, lb, ha, hb;
-        upk(gl[j / 2], la, lb);
-        upk(gh[j / 2], ha, hb);
-        const float glo = fabsf((j & 1) ? lb : la), ghi = fabsf((j & 1) ? hb : ha);
-        const float t = __fmul_rn(__fadd_rn(glo, ghi), 0.5f);            // the threshold between them
-        const uint32_t tb = __float_as_uint(t);
-        const float hu = __uint_as_float((tb & 0x7f800000u) - (24u << 23)); // half spacing above t
-        const float hl = (tb & 0x007fffffu) ? hu : __fmul_rn(hu, 0.5f);     // ... below t
-        const float r = __fmaf_rn(-t, S, fabsf(y[j]));
-        uint32_t mag;
-        if (r > __fmul_rn(hu, S)) mag = cb & 7u;
-        else if (r < -__fmul_rn(hl, S)) mag = ca & 7u;
-        else mag = ((ca & 7u) & 1u) ? (cb & 7u) : (ca & 7u);              // tie: even magnitude code
-        out = (out & ~(0xfu << (4 * j))) | (((ca & 8u) | mag) << (4 * j));
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+        float S;
+        if (FMT == kUE4M3) S = c < 127 ? __fmul_rn(ue4m3_decode((uint32_t)c), G) : __uint_as_float(0x7fc00000u);
+        else S = c < 255 ? __fmul_rn(ue5m3_decode((uint32_t)c), G) : __uint_as_float(0x7fc00000u);
+        float R;
+        if (S == 0.0f) R = 0.0f;
+        else if (S >= kDivLo && S <= kDivHi) R = __frcp_rn(S);
+        else R = __uint_as_float(0x7f800000u);
+        tab[c] = make_float2(S, R);
     }
-    return out;
 }
 
-// Scales of the NB blocks of a unit: codes, S and the bracket of 1/S.  The UE4M3
-// rule runs on two blocks at a time with two-wide instructions.
+// Scales of the NB blocks of a unit ("max" rule): scale bytes, S and R =
+// fp32(1/S).  E8M0: S = 2^(floor(log2 m) - 2), R exact.  UE4M3 / UE5M3: the
+// byte is the code nearest the correctly rounded quotient fp32(m / fp32(6G))
+// (two blocks per instruction), S and R come from the table.  Returns false
+// when some block must divide its elements: fp32(6G) or S outside the range
+// of the remainder correction, or a quotient m / S beyond 2^60.
 template <int FMT, int NB>
-__device__ __forceinline__ bool unit_scales(const float (&m)[NB], const ScaleConsts& kc, uint32_t (&code)[NB],
-                                            float (&S)[NB], float (&rlo)[NB], float (&rhi)[NB])
+__device__ __forceinline__ bool unit_scales(const float (&m)[NB], const ScaleConsts& kc, const float2* tab,
+                                            uint32_t (&code)[NB], float (&S)[NB], float (&R)[NB])
 {
-    bool exact = true;
-    if constexpr (FMT == kUE4M3 && NB >= 2) {
-#pragma unroll
-        for (int bi = 0; bi < NB; bi += 2) {
-            exact = block_scale_ue4m3_pair(m[bi], m[bi + 1], kc, code[bi], code[bi + 1], S[bi], S[bi + 1], rlo[bi],
-                                           rlo[bi + 1], rhi[bi], rhi[bi + 1]) && exact;
-        }
-    } else {
+    if constexpr (FMT == kE8M0) {
 #pragma unroll
         for (int bi = 0; bi < NB; ++bi) {
-            bool ok;
-            code[bi] = block_scale<FMT>(m[bi], kc, S[bi], rlo[bi], rhi[bi], ok);
-            exact = exact && ok;
+            code[bi] = e8m0_from_amax(m[bi]);
+            S[bi] = e8m0_decode(code[bi]);
+            R[bi] = e8m0_inverse(code[bi]);
         }
+        return true;
+    } else {
+        bool fast = kc.denom_ok;
+#pragma unroll
+        for (int bi = 0; bi < NB; bi += 2) {
+            const float m1 = bi + 1 < NB ? m[bi + 1] : m[bi];
+            float s0, s1;
+            if (kc.denom_ok) {
+                upk(div2_cr(pk(m[bi], m1), pk(kc.rdenom, kc.rdenom), pk(-kc.denom, -kc.denom)), s0, s1);
+            } else {
+                s0 = __fdiv_rn(m[bi], kc.denom);
+                s1 = __fdiv_rn(m1, kc.denom);
+            }
+            uint32_t c0, c1;
+            if constexpr (FMT == kUE4M3) {
+                const uint32_t cc = ue4m3_encode2(s0, s1);
+                c0 = cc & 0xffu;
+                c1 = cc >> 8;
+            } else {
+                c0 = ue5m3_encode(s0);
+                c1 = ue5m3_encode(s1);
+            }
+            code[bi] = c0;
+            if (bi + 1 < NB) code[bi + 1] = c1;
+        }
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) {
+            const float2 e = tab[code[bi]];
+            S[bi] = e.x;
+            R[bi] = e.y;
+            fast = fast && (__fmul_rn(m[bi], e.y) <= kQuotMax);
+        }
+        return fast;
     }
-    return exact;
+}
+
+// Largest dequantized magnitude of a block, |v| of its maximum m: the grid
+// value that fp32(m / S) rounds to, times S.  For a UE scale with a normal
+// code (byte >= 8: 3 significant bits), when fp32(6G) and S are in the
+// normal range (`fast`), decode(s) is within 2^-4 (relative) of m / fp32(6G),
+// so m / S lies in [5.6, 6.5] and always rounds to 6.  E8M0 scales are powers
+// of two, so m * (1/S) is the exact quotient.  Other UE blocks divide.
+template <int FMT>
+__device__ __forceinline__ float block_vmax(float m, float S, float r_mid, uint32_t code, bool fast)
+{
+    if (S == 0.0f) return 0.0f;
+    if constexpr (FMT == kE8M0) {
+        return __fmul_rn(e2m1_grid_value(__fmul_rn(m, r_mid)), S);
+    } else {
+        if (fast && code >= 8u) return __fmul_rn(6.0f, S);
+        return __fmul_rn(e2m1_grid_value(__fdiv_rn(m, S)), S);
+    }
 }
 
 // ---------------------------------------------------------------- quantize
@@ -359,7 +405,8 @@ struct QuantParams {
 
 template <int FMT, int B, int K, bool MSE>
 __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
-                                              int lane, const ScaleConsts& kc, double (&acc)[4])
+                                              int lane, const ScaleConsts& kc, const float2* tab, float nz,
+                                              double (&acc)[3])
 {
     using S = UnitShape<B, K>;
     constexpr int NB = S::NB, BE = S::BE;
@@ -368,39 +415,39 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
 
     float m[NB];
-    block_max<B, K>(v, m);
+    if constexpr (K == 0) block_max_words<B>(w, m);
+    else block_max<B, K>(v, m);
 
-    float sc[NB], rlo[NB], rhi[NB];
+    float sc[NB], rm[NB];
     uint32_t code[NB];
-    const bool exact = unit_scales<FMT, NB>(m, kc, code, sc, rlo, rhi);
+    const bool exact = unit_scales<FMT, NB>(m, kc, tab, code, sc, rm);
 
     uint32_t cw[EPT / 8];
     if constexpr (FMT == kE8M0) {
-        // S is a power of two: y * (1/S) is exactly the quotient.
+        // S is a power of two: y * (1/S) is the quotient itself.
 #pragma unroll
         for (int k = 0; k < EPT / 8; ++k) {
-            const f32x2 r = pk(rlo[(8 * k) / BE], rlo[(8 * k) / BE]);
+            const f32x2 r = pk(rm[(8 * k) / BE], rm[(8 * k) / BE]);
             cw[k] = pack_pairs(mul2(v[4 * k], r), mul2(v[4 * k + 1], r), mul2(v[4 * k + 2], r),
                                mul2(v[4 * k + 3], r));
         }
     } else {
+        if (exact) {
+            // correctly rounded quotients y / S (remainder correction), then the
+            // hardware E2M1 rounding (nearest, ties to the even code, saturating)
 #pragma unroll
-        for (int k = 0; k < EPT / 8; ++k) {
-            const int bi = (8 * k) / BE;
-            const f32x2 rl = pk(rlo[bi], rlo[bi]), rh = pk(rhi[bi], rhi[bi]);
-            const uint32_t a = pack_pairs(mul2(v[4 * k], rl), mul2(v[4 * k + 1], rl), mul2(v[4 * k + 2], rl),
-                                          mul2(v[4 * k + 3], rl));
-            const uint32_t b = pack_pairs(mul2(v[4 * k], rh), mul2(v[4 * k + 1], rh), mul2(v[4 * k + 2], rh),
-                                          mul2(v[4 * k + 3], rh));
-            // a quotient on (or within the bracket of) a threshold: settle it exactly
-            cw[k] = (a == b) ? a : resolve_ties(a, b, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], sc[bi]);
-        }
-        if (!exact) {
-            // extreme scales (S or 1/S not a normal float): correctly rounded divisions
+            for (int k = 0; k < EPT / 8; ++k) {
+                const int bi = (8 * k) / BE;
+                const f32x2 R2 = pk(rm[bi], rm[bi]), nS2 = pk(-sc[bi], -sc[bi]);
+                cw[k] = pack_pairs(div2_cr(v[4 * k], R2, nS2), div2_cr(v[4 * k + 1], R2, nS2),
+                                   div2_cr(v[4 * k + 2], R2, nS2), div2_cr(v[4 * k + 3], R2, nS2));
+            }
+        } else {
+            // extreme scales: correctly rounded divisions
 #pragma unroll
             for (int k = 0; k < EPT / 8; ++k) {
                 const float s = sc[(8 * k) / BE];
-                if (s != 0.0f) cw[k] = pack_pairs_div(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], s);
+                cw[k] = s != 0.0f ? pack_pairs_div(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], s) : 0u;
             }
         }
         // zero-rounded blocks store plain 0x0 nibbles
@@ -409,50 +456,45 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
             if (sc[(8 * k) / BE] == 0.0f) cw[k] = 0u;
     }
 
-    // ---- fused MSE (three-term split of "Finer is better?"): v_i = decode(code_i) * S
+    // ---- fused MSE (three-term split of "Finer is better?"): v_i = fp32(decode(code_i) * S)
     if constexpr (MSE) {
+        const f32x2 nz2 = pk(nz, nz);            // -0: fma(g, S, -0) is the rounded product fp32(g S)
+        float tot = 0.0f, mx = 0.0f, zr = 0.0f;
 #pragma unroll
         for (int bi = 0; bi < NB; ++bi) {
             const f32x2 s2 = pk(sc[bi], sc[bi]);
             f32x2 sum = pk(0.0f, 0.0f);
-            float vmax = 0.0f;
 #pragma unroll
             for (int k = bi * BE / 8; k < (bi + 1) * BE / 8; ++k) {
                 f32x2 g[4];
                 decode8(cw[k], g);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const f32x2 d = sub2(v[4 * k + j], mul2_rounded(g[j], s2));   // y - fp32(g S)
+                    const f32x2 d = sub2(v[4 * k + j], fma2(g[j], s2, nz2));     // y - fp32(g S)
                     sum = fma2(d, d, sum);
-                    float a, b;
-                    upk(g[j], a, b);
-                    vmax = amax3(a, b, vmax);
                 }
             }
-            vmax = __fmul_rn(vmax, sc[bi]);                          // largest |v| of the block
             float se, so;
             upk(sum, se, so);
             float s = __fadd_rn(se, so);
-            if constexpr (S::LPB > 1) {
-                s = group_sum<S::LPB>(s);
-                vmax = group_max<S::LPB>(vmax);
-            }
+            if constexpr (S::LPB > 1) s = group_sum<S::LPB>(s);
+            const float vmax = block_vmax<FMT>(m[bi], sc[bi], rm[bi], code[bi], exact);
             const int64_t eb = u * EPT + (int64_t)bi * BE;
             const bool leader = (S::LPB == 1) || ((lane % S::LPB) == 0);
             if (leader && eb < p.n) {
                 if (p.block_mse) p.block_mse[eb / B] = __fmul_rn(s, 1.0f / (float)B);
-                acc[0] += (double)s;
+                tot = __fadd_rn(tot, s);
                 if (vmax == 0.0f) {
-                    acc[3] += (double)s;
+                    zr = __fadd_rn(zr, s);                  // every v of the block is 0
                 } else {
-                    // the block maximum rounds to the largest |v| of the block
-                    const float dm = __fsub_rn(m[bi], vmax);
-                    const float emax = __fmul_rn(dm, dm);
-                    acc[2] += (double)emax;
-                    acc[1] += (double)s - (double)emax;
+                    const float dm = __fsub_rn(m[bi], vmax);   // the maximum rounds to the largest |v|
+                    mx = __fmaf_rn(dm, dm, mx);
                 }
             }
         }
+        acc[0] += (double)tot;
+        acc[1] += (double)mx;
+        if (zr != 0.0f) acc[2] += (double)zr;
     }
 
     // ---- stores
@@ -504,15 +546,22 @@ __global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantPa
     float G = 1.0f;
     if (FMT != kE8M0 && p.gsrc != nullptr) G = *p.gsrc;
     const ScaleConsts kc = scale_consts(G);
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    __shared__ float2 tab[256];                 // UE scales {S, 1/S} by code
+    if constexpr (FMT != kE8M0) fill_scale_table<FMT>(tab, G);
+    __syncthreads();
+    // -0.0f from a value the compiler cannot see (n >= 0 at run time): an
+    // fma with it rounds a product on its own and cannot be merged with the
+    // subtraction that follows.
+    const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
+    double acc[3] = {0.0, 0.0, 0.0};        // squared errors: all, block maxima, zero-rounded blocks
 
     stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
                  [&](int64_t t, int s) {
                      uint32_t w[EPT / 2];
                      ring.read(s, 0, w);
-                     quantize_unit<FMT, B, K, MSE>(p, t * 32 + lane, w, lane, kc, acc);
+                     quantize_unit<FMT, B, K, MSE>(p, t * 32 + lane, w, lane, kc, tab, nz, acc);
                  });
-    if constexpr (MSE) cta_partials(acc[0], acc[1], acc[2], acc[3], p.partials);
+    if constexpr (MSE) cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
 }
 
 // ---------------------------------------------------------------- per-tensor amax
@@ -925,33 +974,27 @@ static __global__ void __launch_bounds__(kThreads) e2m1_encode_kernel(const floa
     }
 }
 
-// Scale codes one value at a time through the quantizer's own block-scale
-// routines with 6 G = 1: UE formats give the code nearest to s, E8M0 the byte
-// of a block whose maximum is s.  UE4M3 goes through the paired routine the
-// quantizer uses for two blocks (values i and i + 1 form a pair).
+// Scale codes one value at a time through the quantizer's own encoders: UE
+// formats give the code nearest to s (the quantizer applies the same encoder,
+// two values at a time for UE4M3, to the correctly rounded m / fp32(6G)),
+// E8M0 the byte of a block whose maximum is s.
 static __global__ void __launch_bounds__(kThreads) scale_encode_kernel(const float* __restrict__ s, int64_t n,
                                                                       int fmt, uint8_t* __restrict__ out)
 {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    ScaleConsts k1;
-    k1.G = 1.0f;
-    k1.denom = 1.0f;
-    k1.denom_ok = true;
-    k1.rd_lo = kBracketLo;
-    k1.rd_hi = kBracketHi;
     for (int64_t i = 2 * ((int64_t)blockIdx.x * kThreads + threadIdx.x); i < n; i += 2 * stride) {
         const float s0 = s[i], s1 = (i + 1 < n) ? s[i + 1] : 0.0f;
-        float S0, S1, a0, a1, b0, b1;
-        bool ok;
         uint32_t c0, c1;
         if (fmt == kE8M0) {
-            c0 = block_scale<kE8M0>(s0, k1, S0, a0, b0, ok);
-            c1 = block_scale<kE8M0>(s1, k1, S1, a1, b1, ok);
+            c0 = e8m0_from_amax(s0);
+            c1 = e8m0_from_amax(s1);
         } else if (fmt == kUE4M3) {
-            block_scale_ue4m3_pair(s0, s1, k1, c0, c1, S0, S1, a0, a1, b0, b1);
+            const uint32_t cc = ue4m3_encode2(s0, s1);
+            c0 = cc & 0xffu;
+            c1 = cc >> 8;
         } else {
-            c0 = block_scale<kUE5M3>(s0, k1, S0, a0, b0, ok);
-            c1 = block_scale<kUE5M3>(s1, k1, S1, a1, b1, ok);
+            c0 = ue5m3_encode(s0);
+            c1 = ue5m3_encode(s1);
         }
         out[i] = (uint8_t)c0;
         if (i + 1 < n) out[i + 1] = (uint8_t)c1;
