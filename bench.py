@@ -33,7 +33,7 @@ if ROOT not in sys.path:
 METRIC = "G elements/s and achieved HBM GB/s (% of B200 peak) for rotate+FP4 quantize"
 SPEC_HBM_GBS = 8000.0
 E8, U4, U5 = 0, 1, 2
-NONE, COMP, GIVEN = 0, 1, 2
+NONE, COMP, GIVEN, FROM_AMAX = 0, 1, 2, 3
 
 
 # --------------------------------------------------------------------------- args / dist
@@ -141,39 +141,40 @@ class Pipeline:
             b = dict(
                 codes=torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
                 scales=torch.empty((rows, cols // block), dtype=torch.uint8, device=device),
-                amax=torch.empty((1,), dtype=torch.float32, device=device),
-                gscale=torch.empty((1,), dtype=torch.float32, device=device),
+                gscale=torch.empty((2,), dtype=torch.float32, device=device),     # [amax, G]
                 deq=torch.empty((rows, cols), dtype=torch.bfloat16, device=device),
                 bm=torch.empty((rows, cols // block), dtype=torch.float32, device=device),
                 terms=torch.empty((4,), dtype=torch.float64, device=device),
-                ws=torch.empty((fq.fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
+                ws=torch.zeros((fq.fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
                                device=device),
             )
             self.bufs.append(b)
             p = {k: v.data_ptr() for k, v in b.items()}
             comp = gmode == COMP
-            g = p["gscale"] if comp else None
+            # per-tensor scale: the amax pass writes gscale[0]; the quantizer derives G from it
+            # (FROM_AMAX) and writes it to gscale[1], where dequantize and block MSE read it
+            gq = p["gscale"] if comp else None
+            g = p["gscale"] + 4 if comp else None
             seq = []
             if comp:
-                seq.append(("amax", L.fp4q_tensor_amax, (x.data_ptr(), rows, cols, rot, p["amax"], sh)))
-                seq.append(("global_scale", L.fp4q_global_scale, (p["amax"], p["gscale"], sh)))
-            gm = GIVEN if comp else NONE
+                seq.append(("amax", L.fp4q_tensor_amax, (x.data_ptr(), rows, cols, rot, p["gscale"], sh)))
+            gm = FROM_AMAX if comp else NONE
             if separate_mse:
                 seq.append(("quantize", L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot, gm,
-                                                          p["codes"], p["scales"], g, sh)))
+                                                          p["codes"], p["scales"], gq, sh)))
                 seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
                                                             fmt, block, rot, p["bm"], p["terms"], p["ws"],
                                                             b["ws"].numel(), sh)))
             else:
                 seq.append(("quantize_mse", L.fp4q_quantize_mse,
-                            (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], g, p["bm"],
+                            (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], gq, p["bm"],
                              p["terms"], p["ws"], b["ws"].numel(), sh)))
             seq.append(("dequantize", L.fp4q_dequantize, (p["codes"], p["scales"], g, rows, cols, fmt, block, 0,
                                                           0, p["deq"], sh)))
             self.calls.append(seq)
         self.elements = sum(x.numel() for _, x, *_ in items)
-        # kernels per step: amax + G (per-tensor scale), quantize (+MSE) and the MSE finalize, dequantize
-        self.launches_per_step = sum(3 + (2 if gm == COMP else 0) + (1 if separate_mse else 0)
+        # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel), [block MSE], dequantize
+        self.launches_per_step = sum(2 + (1 if gm == COMP else 0) + (1 if separate_mse else 0)
                                      for *_, gm in items)
         self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
 

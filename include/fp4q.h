@@ -76,7 +76,10 @@ typedef enum {
 typedef enum {
     FP4Q_GLOBAL_NONE = 0,      /* G = 1 (always for E8M0; plain UE4M3 / UE5M3)  */
     FP4Q_GLOBAL_COMPUTE = 1,   /* G = amax(|y|)/(6*448) (1 if amax = 0), written to *gscale */
-    FP4Q_GLOBAL_GIVEN = 2      /* G read from *gscale (must be finite and > 0)  */
+    FP4Q_GLOBAL_GIVEN = 2,     /* G read from *gscale (must be finite and > 0)  */
+    FP4Q_GLOBAL_FROM_AMAX = 3  /* gscale[0] holds amax(|y|) on entry (for instance from
+                                  fp4q_tensor_amax); G = amax/(6*448) (1 if amax = 0) is
+                                  computed by the call and written to gscale[1]         */
 } fp4q_global_mode;
 
 typedef enum {
@@ -96,7 +99,9 @@ typedef enum {
  *  gmode   fp4q_global_mode; must be FP4Q_GLOBAL_NONE for E8M0.
  *  codes   out: rows*cols/2 bytes.  scales: out, rows*cols/block bytes.
  *  gscale  1 float: written in COMPUTE mode, read in GIVEN mode, ignored (may
- *          be NULL) in NONE mode.
+ *          be NULL) in NONE mode.  FROM_AMAX: 2 floats, the tensor's maximum
+ *          |y| in gscale[0] (read) and G in gscale[1] (written); same codes,
+ *          scales and G as COMPUTE without a pass over x for the maximum.
  * Per block: m = max |y|; E8M0 S = 2^(floor(log2 m)-2); UE4M3/UE5M3
  * s = nearest code to fp32(m / fp32(6 G)) (ties to even, saturating), S =
  * fp32(decode(s) G).  Each nibble is the E2M1 value nearest to fp32(y / S)
@@ -148,7 +153,15 @@ FP4Q_API int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const 
  *                 of its dequantized values are 0; the block max is an element
  *                 of largest |y|.
  *  workspace    device scratch of at least fp4q_block_mse_workspace_size()
- *               bytes, 8-byte aligned; its contents on entry do not matter.
+ *               bytes, 8-byte aligned.  Its first 16 bytes hold the counter
+ *               through which the kernel's CTAs find the last one to finish
+ *               (which then sums the per-CTA partials): they must be zero
+ *               before the first call that uses the workspace, and every
+ *               completed call leaves them zero.  Allocate it zero-filled once
+ *               and reuse it for tensors of any size (at least as large as
+ *               the workspace size each needs); the rest is overwritten by
+ *               each call.  Calls that share a workspace must not run at the
+ *               same time.
  * The per-tensor sums use a fixed reduction order (deterministic run to run).
  */
 FP4Q_API int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,
@@ -164,7 +177,9 @@ FP4Q_API int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* 
  * maximum's error is taken against the largest dequantized magnitude of the
  * block (the value the maximum rounds to), the per-block sums are fp32 and the
  * tensor terms fp64 in a fixed order.  workspace: at least
- * fp4q_block_mse_workspace_size() bytes.
+ * fp4q_block_mse_workspace_size() bytes, with the zeroed completion counter
+ * described at fp4q_block_mse.  gmode may be FP4Q_GLOBAL_FROM_AMAX as for
+ * fp4q_quantize.
  */
 FP4Q_API int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
                                int gmode, uint8_t* codes, uint8_t* scales, float* gscale,
@@ -172,7 +187,8 @@ FP4Q_API int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fm
                                void* stream);
 
 /* Bytes of device workspace fp4q_block_mse and fp4q_quantize_mse need for this
- * shape (host only; at most 128 KiB). */
+ * shape (host only; at most 128 KiB + 16): the completion counter and the
+ * per-CTA partials. */
 FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block);
 
 /*
@@ -192,8 +208,9 @@ FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int bl
  *  - Setup: the first call on each device (with that device current) looks
  *    up the buffer's device address with cudaGetSymbolAddress and caches it.
  *    Make that first call before any stream capture begins on the device.
- *  - Nothing needs to start at zero: every launched CTA overwrites its own
- *    slot before the final reduction reads it.
+ *  - The buffer ends with the completion counter of the in-kernel reduction
+ *    (see fp4q_block_mse): it is zero when the library is loaded and every
+ *    completed call leaves it zero; the partials are overwritten by each call.
  *  - One buffer per device: two calls in flight at the same time on one
  *    device (on different streams, or from different host threads without
  *    ordering) race on it and give wrong terms.  Calls ordered on one stream

@@ -21,12 +21,13 @@ LIB_PATH = os.path.join(_PKG, "libfp4q.so")
 # enums of include/fp4q.h
 FP4Q_OK = 0
 FP4Q_SCALE_E8M0, FP4Q_SCALE_UE4M3, FP4Q_SCALE_UE5M3 = 0, 1, 2
-FP4Q_GLOBAL_NONE, FP4Q_GLOBAL_COMPUTE, FP4Q_GLOBAL_GIVEN = 0, 1, 2
+FP4Q_GLOBAL_NONE, FP4Q_GLOBAL_COMPUTE, FP4Q_GLOBAL_GIVEN, FP4Q_GLOBAL_FROM_AMAX = 0, 1, 2, 3
 FP4Q_OUT_BF16, FP4Q_OUT_F32 = 0, 1
 
 _FMT_NAMES = {"e8m0": FP4Q_SCALE_E8M0, "mxfp4": FP4Q_SCALE_E8M0, "ue4m3": FP4Q_SCALE_UE4M3,
               "nvfp4": FP4Q_SCALE_UE4M3, "ue5m3": FP4Q_SCALE_UE5M3}
-_GMODE_NAMES = {"none": FP4Q_GLOBAL_NONE, "compute": FP4Q_GLOBAL_COMPUTE, "given": FP4Q_GLOBAL_GIVEN}
+_GMODE_NAMES = {"none": FP4Q_GLOBAL_NONE, "compute": FP4Q_GLOBAL_COMPUTE, "given": FP4Q_GLOBAL_GIVEN,
+                "from_amax": FP4Q_GLOBAL_FROM_AMAX}
 
 
 class Fp4qError(RuntimeError):
@@ -127,8 +128,12 @@ def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
         codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
     if scales is None:
         scales = torch.empty((rows, cols // block if block else 0), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode == FP4Q_GLOBAL_FROM_AMAX:
+        raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
     if gscale is None and gmode != FP4Q_GLOBAL_NONE:
         gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    if gmode == FP4Q_GLOBAL_FROM_AMAX and gscale.numel() < 2:
+        raise ValueError("from_amax mode needs gscale with 2 floats: [amax in, G out]")
     _need_cuda(codes, scales, gscale)
     st = lib().fp4q_quantize(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(codes), _ptr(scales),
                             _ptr(gscale), _stream(stream))
@@ -195,7 +200,7 @@ def fp4q_block_mse(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
         terms = torch.empty((4,), dtype=torch.float64, device=dev)
     ws = fp4q_block_mse_workspace_size(rows, cols, block)
     if workspace is None:
-        workspace = torch.empty((ws,), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros((ws,), dtype=torch.uint8, device=dev)
     st = lib().fp4q_block_mse(_ptr(x), _ptr(codes), _ptr(scales), _ptr(gscale), rows, cols, _fmt(fmt),
                              block, rot, _ptr(block_mse), _ptr(terms), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream))
@@ -242,14 +247,18 @@ def fp4q_quantize_mse(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="non
         codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
     if scales is None:
         scales = torch.empty((rows, cols // block if block else 0), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode == FP4Q_GLOBAL_FROM_AMAX:
+        raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
     if gscale is None and gmode != FP4Q_GLOBAL_NONE:
         gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    if gmode == FP4Q_GLOBAL_FROM_AMAX and gscale.numel() < 2:
+        raise ValueError("from_amax mode needs gscale with 2 floats: [amax in, G out]")
     if block_mse is None and want_block_mse:
         block_mse = torch.empty((rows, cols // block if block else 0), dtype=torch.float32, device=dev)
     if terms is None:
         terms = torch.empty((4,), dtype=torch.float64, device=dev)
     if workspace is None:
-        workspace = torch.empty((fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
+        workspace = torch.zeros((fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
                                 device=dev)
     _need_cuda(codes, scales, gscale, block_mse, terms, workspace)
     st = lib().fp4q_quantize_mse(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(codes), _ptr(scales),

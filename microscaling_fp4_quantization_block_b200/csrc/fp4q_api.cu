@@ -49,6 +49,31 @@ void rotation_constants(int rot, float* hi, float* lo)
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
+// MSE workspace: a 16-byte slot whose first word is the completion counter of
+// the in-kernel reduction (at a fixed place, so one workspace serves tensors of
+// any size), then partial_slots(n) rows of 4 doubles.
+constexpr size_t kCounterBytes = 16;
+unsigned int* mse_counter(void* workspace) { return static_cast<unsigned int*>(workspace); }
+double* mse_partials(void* workspace)
+{
+    return reinterpret_cast<double*>(static_cast<char*>(workspace) + kCounterBytes);
+}
+
+bool valid_gmode(int gmode)
+{
+    return gmode == FP4Q_GLOBAL_NONE || gmode == FP4Q_GLOBAL_COMPUTE || gmode == FP4Q_GLOBAL_GIVEN ||
+           gmode == FP4Q_GLOBAL_FROM_AMAX;
+}
+
+// Per-tensor scale source of the quantize kernels for gmode: G itself (GIVEN,
+// and COMPUTE after the amax pass), or the tensor maximum in gscale[0] with G
+// written to gscale[1] (FROM_AMAX).
+void set_global(int gmode, float* gscale, const float** gsrc, float** gdst)
+{
+    *gsrc = gmode == FP4Q_GLOBAL_NONE ? nullptr : gscale;
+    *gdst = gmode == FP4Q_GLOBAL_FROM_AMAX ? gscale + 1 : nullptr;
+}
+
 // amax(|y|) of the tensor into *dst (fp32 bits, via atomicMax on a zeroed slot).
 cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStream_t s)
 {
@@ -65,9 +90,10 @@ cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStre
 // ---- fixed scratch of fp4q_block_mse_noalloc
 // Per-CTA MSE partials for callers that cannot allocate a workspace: one
 // static device buffer per device, 4096 slots of 4 doubles (128 KiB), which is
-// the most partial slots any launch uses (the MSE kernel caps its grid there).
+// the most partial slots any launch uses (the MSE kernel caps its grid there),
+// followed by the completion counter (zero at load, left zero by every call).
 constexpr int kNoAllocSlots = kMaxPartialCtas;
-static __device__ __align__(256) double g_noalloc_partials[kNoAllocSlots * 4];
+static __device__ __align__(256) double g_noalloc_partials[kNoAllocSlots * 4 + 2];   // + completion counter
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
@@ -116,8 +142,7 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
     int64_t n = 0;
     int st = check_shape(rows, cols, fmt, block, rot, &n);
     if (st) return st;
-    if (gmode != FP4Q_GLOBAL_NONE && gmode != FP4Q_GLOBAL_COMPUTE && gmode != FP4Q_GLOBAL_GIVEN)
-        return FP4Q_ERR_UNSUPPORTED;
+    if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
     if (gmode != FP4Q_GLOBAL_NONE) {
         if (!gscale) return FP4Q_ERR_NULL;
@@ -134,13 +159,19 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
         global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
         if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     }
-    if (n == 0) return FP4Q_OK;
+    if (n == 0) {
+        if (gmode == FP4Q_GLOBAL_FROM_AMAX) {
+            global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale + 1);
+            return cuda_status(cudaGetLastError());
+        }
+        return FP4Q_OK;
+    }
     QuantParams p{};
     p.x = static_cast<const uint16_t*>(x);
     p.n = n;
     p.codes = codes;
     p.scales = scales;
-    p.gsrc = (gmode == FP4Q_GLOBAL_NONE) ? nullptr : gscale;
+    set_global(gmode, gscale, &p.gsrc, &p.gdst);
     rotation_constants(rot, &p.c_hi, &p.c_lo);
     return cuda_status(launch_quantize(fmt, block, rot, false, p, nullptr, s));
 }
@@ -152,8 +183,7 @@ int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int bl
     int64_t n = 0;
     int st = check_shape(rows, cols, fmt, block, rot, &n);
     if (st) return st;
-    if (gmode != FP4Q_GLOBAL_NONE && gmode != FP4Q_GLOBAL_COMPUTE && gmode != FP4Q_GLOBAL_GIVEN)
-        return FP4Q_ERR_UNSUPPORTED;
+    if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
     if (gmode != FP4Q_GLOBAL_NONE) {
         if (!gscale) return FP4Q_ERR_NULL;
@@ -174,22 +204,26 @@ int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int bl
         global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
         if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     }
-    double* partials = static_cast<double*>(workspace);
-    int grid = 0;
-    if (n > 0) {
-        QuantParams p{};
-        p.x = static_cast<const uint16_t*>(x);
-        p.n = n;
-        p.codes = codes;
-        p.scales = scales;
-        p.gsrc = (gmode == FP4Q_GLOBAL_NONE) ? nullptr : gscale;
-        p.block_mse = block_mse;
-        p.partials = partials;
-        rotation_constants(rot, &p.c_hi, &p.c_lo);
-        if (launch_quantize(fmt, block, rot, true, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (n == 0) {
+        if (gmode == FP4Q_GLOBAL_FROM_AMAX) {
+            global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale + 1);
+            if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+        }
+        return cuda_status(cudaMemsetAsync(terms, 0, 4 * sizeof(double), s));
     }
-    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
-    return cuda_status(cudaGetLastError());
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.n = n;
+    p.codes = codes;
+    p.scales = scales;
+    set_global(gmode, gscale, &p.gsrc, &p.gdst);
+    p.block_mse = block_mse;
+    p.partials = mse_partials(workspace);
+    p.done = mse_counter(workspace);
+    p.terms = terms;
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
+    int grid = 0;
+    return cuda_status(launch_quantize(fmt, block, rot, true, p, &grid, s));
 }
 
 int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)
@@ -237,7 +271,7 @@ size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block)
     (void)block;
     if (rows < 0 || cols < 0) return 0;
     if (cols != 0 && rows > INT64_MAX / 4 / cols) return 0;
-    return (size_t)partial_slots(rows * cols) * 4 * sizeof(double);
+    return (size_t)partial_slots(rows * cols) * 4 * sizeof(double) + kCounterBytes;
 }
 
 int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, const float* gscale,
@@ -256,23 +290,21 @@ int fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales, c
     if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
     if (ws_bytes < fp4q_block_mse_workspace_size(rows, cols, block)) return FP4Q_ERR_WORKSPACE;
     cudaStream_t s = as_stream(stream);
-    double* partials = static_cast<double*>(workspace);
+    if (n == 0) return cuda_status(cudaMemsetAsync(terms, 0, 4 * sizeof(double), s));
+    MseParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = codes;
+    p.scales = scales;
+    p.gsrc = gscale;
+    p.n = n;
+    p.fmt = fmt;
+    p.block_mse = block_mse;
+    p.partials = mse_partials(workspace);
+    p.done = mse_counter(workspace);
+    p.terms = terms;
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
     int grid = 0;
-    if (n > 0) {
-        MseParams p{};
-        p.x = static_cast<const uint16_t*>(x);
-        p.codes = codes;
-        p.scales = scales;
-        p.gsrc = gscale;
-        p.n = n;
-        p.fmt = fmt;
-        p.block_mse = block_mse;
-        p.partials = partials;
-        rotation_constants(rot, &p.c_hi, &p.c_lo);
-        if (launch_block_mse(block, rot, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
-    }
-    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_block_mse(block, rot, p, &grid, s));
 }
 
 int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* stream)
@@ -319,23 +351,22 @@ int fp4q_block_mse_noalloc(const void* x, const uint8_t* codes, const uint8_t* s
     st = noalloc_partials_for_current_device(&partials);
     if (st) return st;
     cudaStream_t s = as_stream(stream);
+    if (n == 0) return cuda_status(cudaMemsetAsync(terms, 0, 4 * sizeof(double), s));
+    MseParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = codes;
+    p.scales = scales;
+    p.gsrc = gscale;
+    p.n = n;
+    p.fmt = fmt;
+    p.block_mse = block_mse;
+    p.partials = partials;
+    p.done = reinterpret_cast<unsigned int*>(partials + kNoAllocSlots * 4);
+    p.terms = terms;
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
+    // the launch uses at most partial_slots(n) CTAs, checked above to fit the scratch
     int grid = 0;
-    if (n > 0) {
-        MseParams p{};
-        p.x = static_cast<const uint16_t*>(x);
-        p.codes = codes;
-        p.scales = scales;
-        p.gsrc = gscale;
-        p.n = n;
-        p.fmt = fmt;
-        p.block_mse = block_mse;
-        p.partials = partials;
-        rotation_constants(rot, &p.c_hi, &p.c_lo);
-        // the launch uses at most partial_slots(n) CTAs, checked above to fit the scratch
-        if (launch_block_mse(block, rot, p, &grid, s) != cudaSuccess) return FP4Q_ERR_CUDA;
-    }
-    mse_finalize_kernel<<<1, kThreads, 0, s>>>(partials, grid, n, terms);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_block_mse(block, rot, p, &grid, s));
 }
 
 }  // extern "C"

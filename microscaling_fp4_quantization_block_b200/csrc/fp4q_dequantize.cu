@@ -8,11 +8,19 @@ namespace {
 template <int B, int K, bool F32>
 cudaError_t run_dequantize(const DequantParams& p, cudaStream_t s)
 {
-    auto kern = dequantize_kernel<B, K, F32>;
-    const int64_t tile_elems = 32 * DPL;  // 32 lanes x 128 elements
-    const int64_t tiles = (p.n + tile_elems - 1) / tile_elems;
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
-    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+    if constexpr (K <= kDqChunk) {
+        // rotation runs of at most 16: interleaved chunks, fully coalesced stores
+        auto kern = dequantize_il_kernel<B, K, F32>;
+        const int64_t tiles = (p.n + kDqTile - 1) / kDqTile;
+        const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
+        kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+    } else {
+        auto kern = dequantize_kernel<B, K, F32>;
+        const int64_t tile_elems = 32 * DPL;  // 32 lanes x 128 elements
+        const int64_t tiles = (p.n + tile_elems - 1) / tile_elems;
+        const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
+        kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+    }
     return cudaGetLastError();
 }
 

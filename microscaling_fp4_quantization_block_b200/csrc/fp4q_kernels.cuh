@@ -264,6 +264,42 @@ __device__ __forceinline__ void cta_partials(double a0, double a1, double a2, do
     }
 }
 
+// The tensor terms from the per-CTA partials, inside the kernel that wrote
+// them: every CTA counts itself done on a counter (after making its partials
+// visible); the CTA that finishes last sums partials[0..gridDim.x) in index
+// order (deterministic), writes terms[i] = sum / n, and atomicInc's wrap-around
+// leaves the counter at 0 for the next call.  The counter must be 0 when the
+// kernel starts.
+__device__ __forceinline__ void finish_partials(const double* partials, unsigned int* done, int64_t n, double* terms)
+{
+    __shared__ bool last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicInc(done, gridDim.x - 1u) == gridDim.x - 1u;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    __shared__ double red[kWarps][4];
+    double s[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += kThreads)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[k] += __ldcg(partials + (int64_t)i * 4 + k);
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], d);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) red[wid][k] = s[k];
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        double t = 0.0;
+        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
+        terms[threadIdx.x] = t / (double)n;
+    }
+}
+
 // Grid values of the 8 nibbles of a code word as 4 fp32 pairs (exact).
 __device__ __forceinline__ void decode8(uint32_t cw, f32x2 (&g)[4])
 {
@@ -401,6 +437,9 @@ struct QuantParams {
     float c_hi, c_lo;      // 1/sqrt(K) split in two fp32 parts
     float* block_mse;      // fused MSE: n/B floats or nullptr
     double* partials;      // fused MSE: [gridDim.x][4]
+    unsigned int* done;    // fused MSE: completion counter (0 at launch, left 0)
+    double* terms;         // fused MSE: the four tensor terms
+    float* gdst;           // G from the tensor maximum: *gsrc is that maximum, G is written here
 };
 
 template <int FMT, int B, int K, bool MSE>
@@ -544,7 +583,14 @@ __global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantPa
     const XRing ring = warp_ring<XRing>(smem_ring);
 
     float G = 1.0f;
-    if (FMT != kE8M0 && p.gsrc != nullptr) G = *p.gsrc;
+    if (FMT != kE8M0 && p.gsrc != nullptr) {
+        G = *p.gsrc;
+        if (p.gdst != nullptr) {
+            // per-tensor scale from the tensor maximum: amax / (6 * 448), 1 for an all-zero tensor
+            G = G > 0.0f ? __fdiv_rn(G, 2688.0f) : 1.0f;
+            if (blockIdx.x == 0 && threadIdx.x == 0) *p.gdst = G;
+        }
+    }
     const ScaleConsts kc = scale_consts(G);
     __shared__ float2 tab[256];                 // UE scales {S, 1/S} by code
     if constexpr (FMT != kE8M0) fill_scale_table<FMT>(tab, G);
@@ -561,7 +607,10 @@ __global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantPa
                      ring.read(s, 0, w);
                      quantize_unit<FMT, B, K, MSE>(p, t * 32 + lane, w, lane, kc, tab, nz, acc);
                  });
-    if constexpr (MSE) cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
+    if constexpr (MSE) {
+        cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
+        finish_partials(p.partials, p.done, p.n, p.terms);
+    }
 }
 
 // ---------------------------------------------------------------- per-tensor amax
@@ -773,6 +822,171 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
     });
 }
 
+// ---------------------------------------------------------------- dequantize, interleaved chunks
+// For rotation runs of at most 16 elements.  A warp's tile is 32 x 8 chunks
+// of 16 elements; chunk c of lane l holds elements tile + (32 c + l) * 16 ..
+// + 15, so each store instruction of the warp writes 32 consecutive chunks
+// (1 KiB of bf16, 2 KiB of fp32) and every lane's loads and stores are full
+// 32-byte sectors.  A ring stage holds the tile's 2 KiB of codes followed by
+// its scale bytes (4096 / B, at least one 16-byte chunk), copied with 16-byte
+// cp.async; the block scales come from a per-tensor table of the 256 codes.
+constexpr int kDqChunk = 16;
+constexpr int kDqCpt = 8;                                    // chunks per lane per tile
+constexpr int kDqTile = 32 * kDqCpt * kDqChunk;              // 4096 elements
+
+template <int B>
+struct DqStage {
+    static constexpr int CODE_BYTES = kDqTile / 2;
+    static constexpr int SC_RAW = kDqTile / B;               // 16 .. 512 scale bytes per tile
+    static constexpr int SC_BYTES = SC_RAW < 16 ? 16 : SC_RAW;
+    static constexpr int SC_CHUNKS = SC_BYTES / 16;          // 1 .. 32
+    static constexpr int BYTES = CODE_BYTES + SC_BYTES;
+    static constexpr int NSTAGE = kRingBytesPerWarp / BYTES;
+    static_assert(NSTAGE >= 2 && SC_CHUNKS <= 32, "stage layout");
+};
+
+// Copies of tile t into stage s (sb: its shared address); bytes past the end
+// of the codes or scales are zero-filled and never read from global memory.
+template <int B>
+__device__ __forceinline__ void dq_issue(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                         int64_t code_bytes, int64_t scale_bytes, int64_t t, uint32_t sb, int lane)
+{
+    using D = DqStage<B>;
+    const int64_t co = t * (int64_t)D::CODE_BYTES, so = t * (int64_t)D::SC_RAW;
+    if (co + D::CODE_BYTES <= code_bytes && so + D::SC_BYTES <= scale_bytes) {
+#pragma unroll
+        for (int j = 0; j < D::CODE_BYTES / 512; ++j)
+            cp_async16(sb + 16u * (uint32_t)(lane + 32 * j), codes + co + 16 * (lane + 32 * j), 16u);
+        if (lane < D::SC_CHUNKS) cp_async16(sb + D::CODE_BYTES + 16u * lane, scales + so + 16 * lane, 16u);
+    } else {
+#pragma unroll
+        for (int j = 0; j < D::CODE_BYTES / 512; ++j) {
+            const int64_t o = co + 16 * (lane + 32 * j), left = code_bytes - o;
+            const uint32_t cnt = left >= 16 ? 16u : (left > 0 ? (uint32_t)left : 0u);
+            cp_async16(sb + 16u * (uint32_t)(lane + 32 * j), cnt ? (const void*)(codes + o) : (const void*)codes, cnt);
+        }
+        if (lane < D::SC_CHUNKS) {
+            const int64_t o = so + 16 * lane, left = scale_bytes - o;
+            const uint32_t cnt = left >= 16 ? 16u : (left > 0 ? (uint32_t)left : 0u);
+            cp_async16(sb + D::CODE_BYTES + 16u * lane, cnt ? (const void*)(scales + o) : (const void*)scales, cnt);
+        }
+    }
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t smem_addr)
+{
+    uint2 r;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(smem_addr));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t lds_u8(uint32_t smem_addr)
+{
+    uint32_t r;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(r) : "r"(smem_addr));
+    return r;
+}
+
+template <int B, int K, bool F32OUT>
+__global__ void __launch_bounds__(kThreads) dequantize_il_kernel(DequantParams p)
+{
+    static_assert(K == 0 || K == kDqChunk, "interleaved chunks hold rotation runs of at most 16");
+    using D = DqStage<B>;
+    extern __shared__ __align__(128) uint8_t smem_ring[];
+    __shared__ float tab[256];                                   // block scale by code
+    const int lane = threadIdx.x & 31;
+    const float G = (p.fmt != kE8M0 && p.gsrc != nullptr) ? *p.gsrc : 1.0f;
+    for (int c = threadIdx.x; c < 256; c += kThreads) tab[c] = decode_scale((uint32_t)c, p.fmt, G);
+    __syncthreads();
+
+    const int64_t n_tiles = (p.n + kDqTile - 1) / kDqTile;
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem_ring) + (uint32_t)((threadIdx.x >> 5) * kRingBytesPerWarp);
+    const int64_t code_bytes = p.n / 2, scale_bytes = p.n / B;
+    constexpr int NS = D::NSTAGE;
+
+    int64_t t_issue = warp;
+#pragma unroll
+    for (int s = 0; s < NS - 1; ++s) {
+        if (t_issue < n_tiles) dq_issue<B>(p.codes, p.scales, code_bytes, scale_bytes, t_issue, ring + s * D::BYTES, lane);
+        cp_async_commit();
+        t_issue += n_warps;
+    }
+    int stage = 0;
+    for (int64_t t = warp; t < n_tiles; t += n_warps) {
+        const int s_new = stage == 0 ? NS - 1 : stage - 1;
+        if (t_issue < n_tiles) dq_issue<B>(p.codes, p.scales, code_bytes, scale_bytes, t_issue, ring + s_new * D::BYTES, lane);
+        cp_async_commit();
+        t_issue += n_warps;
+        cp_async_wait<NS - 1>();
+        __syncwarp();
+        const uint32_t sb = ring + stage * D::BYTES;
+        const int64_t tile0 = t * kDqTile;
+#pragma unroll 2
+        for (int c = 0; c < kDqCpt; ++c) {
+            const int ch = 32 * c + lane;                        // chunk index in the tile
+            const int64_t e0 = tile0 + (int64_t)ch * kDqChunk;
+            if (e0 >= p.n) break;
+            const uint2 cw = lds64(sb + 8u * (uint32_t)ch);
+            float s0, s1;
+            if constexpr (B == 8) {
+                s0 = tab[lds_u8(sb + D::CODE_BYTES + 2u * ch)];
+                s1 = tab[lds_u8(sb + D::CODE_BYTES + 2u * ch + 1u)];
+            } else {
+                const uint32_t sc = lds_u8(sb + D::CODE_BYTES + (uint32_t)((ch * kDqChunk) / B));
+                s0 = s1 = tab[sc];
+            }
+            f32x2 g[8], v[8];
+            decode8(cw.x, *reinterpret_cast<f32x2(*)[4]>(&g[0]));
+            decode8(cw.y, *reinterpret_cast<f32x2(*)[4]>(&g[4]));
+            const f32x2 S0 = pk(s0, s0), S1 = pk(s1, s1);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = K > 0 ? mul2_rounded(g[j], j < 4 ? S0 : S1) : mul2(g[j], j < 4 ? S0 : S1);
+            if constexpr (K > 0) {
+                fwht_inreg<kDqChunk, K>(v);
+                normalize<kDqChunk>(v, p.c_hi, p.c_lo);
+            }
+            const bool full = e0 + kDqChunk <= p.n;
+            if constexpr (F32OUT) {
+                float* dst = reinterpret_cast<float*>(p.y) + e0;
+                float a[16];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) upk(v[j], a[2 * j], a[2 * j + 1]);
+                if (full) {
+                    stg256(dst, __float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]), __float_as_uint(a[3]),
+                           __float_as_uint(a[4]), __float_as_uint(a[5]), __float_as_uint(a[6]), __float_as_uint(a[7]));
+                    stg256(dst + 8, __float_as_uint(a[8]), __float_as_uint(a[9]), __float_as_uint(a[10]),
+                           __float_as_uint(a[11]), __float_as_uint(a[12]), __float_as_uint(a[13]), __float_as_uint(a[14]),
+                           __float_as_uint(a[15]));
+                } else {
+                    for (int j = 0; j < kDqChunk; ++j)
+                        if (e0 + j < p.n) dst[j] = a[j];
+                }
+            } else {
+                uint32_t o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float a, b;
+                    upk(v[j], a, b);
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+                    o[j] = *reinterpret_cast<uint32_t*>(&hb);
+                }
+                uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.y) + e0);
+                if (full) {
+                    stg256(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                } else {
+                    for (int j = 0; j < 8; ++j)
+                        if (e0 + 2 * j < p.n) dst[j] = o[j];
+                }
+            }
+        }
+        stage = stage + 1 == NS ? 0 : stage + 1;
+        __syncwarp();
+    }
+    cp_async_wait_all();
+}
+
 // ---------------------------------------------------------------- block MSE of given codes
 struct MseParams {
     const uint16_t* x;
@@ -783,6 +997,8 @@ struct MseParams {
     int fmt;
     float* block_mse;      // n/B floats or nullptr
     double* partials;      // [gridDim.x][4]
+    unsigned int* done;    // completion counter (0 at launch, left 0)
+    double* terms;         // the four tensor terms
     float c_hi, c_lo;
 };
 
@@ -928,31 +1144,7 @@ __global__ void __launch_bounds__(kThreads) block_mse_kernel(MseParams p)
         }
     });
     cta_partials(acc_total, acc_nonmax, acc_max, acc_zero, p.partials);
-}
-
-// terms[i] = (sum of partials[*][i]) / n, summed in a fixed order.
-static __global__ void __launch_bounds__(kThreads) mse_finalize_kernel(const double* partials, int nparts,
-                                                                      int64_t n, double* terms)
-{
-    __shared__ double red[kWarps][4];
-    double s[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int i = threadIdx.x; i < nparts; i += kThreads)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) s[k] += partials[(int64_t)i * 4 + k];
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], d);
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (lane == 0)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) red[wid][k] = s[k];
-    __syncthreads();
-    if (threadIdx.x < 4) {
-        double t = 0.0;
-        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
-        terms[threadIdx.x] = n > 0 ? t / (double)n : 0.0;
-    }
+    finish_partials(p.partials, p.done, p.n, p.terms);
 }
 
 // ---------------------------------------------------------------- element codecs

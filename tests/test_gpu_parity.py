@@ -15,7 +15,7 @@ from _helpers import (assert_exact, assert_mse_close, bf16_bits, check_rotated, 
 pytestmark = pytest.mark.gpu
 
 E8, U4, U5 = 0, 1, 2
-NONE, COMP, GIVEN = 0, 1, 2
+NONE, COMP, GIVEN, FROM_AMAX = 0, 1, 2, 3
 
 
 @pytest.fixture(scope="module")
@@ -241,6 +241,58 @@ def test_split_per_tensor_scale_equals_compute_mode(fq):
         assert torch.equal(c1, c2) and torch.equal(s1, s2)
     z = torch.zeros(1, device="cuda")
     assert fq.fp4q_global_scale(z).item() == 1.0
+
+
+@pytest.mark.parametrize("fmt,rot", [(U4, 0), (U4, 32), (U5, 0), (U4, 128)])
+def test_from_amax_mode_equals_compute_mode(fq, fmt, rot):
+    """amax pass -> quantize with G derived in-kernel (FROM_AMAX) gives COMPUTE
+    mode's G, codes and scales; the fused MSE call gives the same terms."""
+    x, _ = workloads.student_t_outliers_bf16(512, 2048, seed=19 + rot)
+    xd = x.cuda()
+    c1, s1, g1 = fq.fp4q_quantize(xd, fmt, 16, rot, COMP)
+    _, _, _, bm1, t1 = fq.fp4q_quantize_mse(xd, fmt, 16, rot, COMP)
+    g2 = torch.empty(2, dtype=torch.float32, device="cuda")
+    fq.fp4q_tensor_amax(xd, rot, amax=g2[:1])
+    c2, s2, _ = fq.fp4q_quantize(xd, fmt, 16, rot, FROM_AMAX, gscale=g2)
+    g3 = g2.clone()
+    g3[1] = -1.0
+    c3, s3, _, bm3, t3 = fq.fp4q_quantize_mse(xd, fmt, 16, rot, FROM_AMAX, gscale=g3)
+    torch.cuda.synchronize()
+    assert g2[1].item() == g1.item() == g3[1].item()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2) and torch.equal(c1, c3) and torch.equal(s1, s3)
+    assert torch.equal(bm1, bm3) and t1.cpu().numpy().tobytes() == t3.cpu().numpy().tobytes()
+
+
+def test_from_amax_mode_empty_and_zero_tensors(fq):
+    for rows, cols in [(0, 64), (4, 64)]:
+        x = torch.zeros((rows, cols), dtype=torch.bfloat16, device="cuda")
+        g = torch.empty(2, dtype=torch.float32, device="cuda")
+        fq.fp4q_tensor_amax(x, 0, amax=g[:1])
+        fq.fp4q_quantize(x, U4, 16, 0, FROM_AMAX, gscale=g)
+        torch.cuda.synchronize()
+        assert g[0].item() == 0.0 and g[1].item() == 1.0
+    with pytest.raises(ValueError):
+        fq.fp4q_quantize(x, U4, 16, 0, FROM_AMAX)
+
+
+def test_mse_workspace_counter_is_left_zero_and_reusable(fq):
+    """The in-kernel reduction's completion counter (first 16 workspace bytes)
+    is zero after every call, so one zero-filled workspace serves many calls of
+    any size: each kernel's terms equal those it gives with a fresh workspace,
+    bit for bit (the fused and the separate kernels sum in different orders)."""
+    big = workloads.gaussian_bf16(1024, 4096, 0.02, seed=31).cuda()
+    small = workloads.gaussian_bf16(16, 512, 0.02, seed=32).cuda()
+    ws = torch.zeros(fq.fp4q_block_mse_workspace_size(1024, 4096, 16), dtype=torch.uint8, device="cuda")
+    for x in (big, small, big, small):
+        c, s, g, bm, t_shared = fq.fp4q_quantize_mse(x, U4, 16, 0, COMP, workspace=ws)
+        _, _, _, _, t_fresh = fq.fp4q_quantize_mse(x, U4, 16, 0, COMP)
+        _, u_fresh = fq.fp4q_block_mse(x, c, s, g, U4, 16, want_block_mse=False)
+        _, u_shared = fq.fp4q_block_mse(x, c, s, g, U4, 16, want_block_mse=False, workspace=ws)
+        torch.cuda.synchronize()
+        assert not ws[:16].any().item(), "completion counter not reset"
+        assert t_shared.cpu().numpy().tobytes() == t_fresh.cpu().numpy().tobytes()
+        assert u_shared.cpu().numpy().tobytes() == u_fresh.cpu().numpy().tobytes()
+        assert np.allclose(t_shared.cpu().numpy(), u_shared.cpu().numpy(), rtol=1e-6, atol=0)
 
 
 FUSED_CASES = [(E8, 32, 0, NONE), (U4, 16, 0, COMP), (U4, 16, 0, NONE), (U4, 8, 0, NONE), (E8, 256, 0, NONE),
