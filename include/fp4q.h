@@ -121,6 +121,16 @@ FP4Q_API int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot
                      void* stream);
 
 /*
+ * fp4q_tensor_amax_accumulate -- *amax = max(*amax, max |y| over the tensor):
+ * the maximum of fp4q_tensor_amax folded into a value already in place, with
+ * no clearing pass.  *amax must hold a non-negative float on entry (0, or the
+ * maximum of other shards of the same tensor, so that shards quantized with
+ * one per-tensor scale share it).  Calls on one slot may run concurrently.
+ */
+FP4Q_API int fp4q_tensor_amax_accumulate(const void* x, int64_t rows, int64_t cols, int rot, float* amax,
+                                         void* stream);
+
+/*
  * fp4q_global_scale -- *gscale = amax / (6 * 448) (correctly rounded fp32), or
  * 1 when amax = 0: the per-tensor scale of COMPUTE mode from an absolute
  * maximum that is already known (for instance one reduced across several

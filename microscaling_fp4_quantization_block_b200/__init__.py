@@ -45,6 +45,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "fp4q_quantize": (I, [P, I64, I64, I, I, I, I, P, P, P, P]),
         "fp4q_tensor_amax": (I, [P, I64, I64, I, P, P]),
+        "fp4q_tensor_amax_accumulate": (I, [P, I64, I64, I, P, P]),
         "fp4q_global_scale": (I, [P, P, P]),
         "fp4q_dequantize": (I, [P, P, P, I64, I64, I, I, I, I, P, P]),
         "fp4q_block_mse": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P, SZ, P]),
@@ -151,6 +152,18 @@ def fp4q_tensor_amax(x: torch.Tensor, rot: int = 0, amax: Optional[torch.Tensor]
         amax = torch.empty((1,), dtype=torch.float32, device=x.device)
     st = lib().fp4q_tensor_amax(_ptr(x), x.shape[0], x.shape[1], rot, _ptr(amax), _stream(stream))
     _check(st, "fp4q_tensor_amax")
+    return amax
+
+
+def fp4q_tensor_amax_accumulate(x: torch.Tensor, amax: torch.Tensor, rot: int = 0, stream=None) -> torch.Tensor:
+    """amax <- max(amax, max |y|) in place (amax: a 1-float CUDA tensor holding a
+    non-negative value, e.g. 0 or the maximum of other shards)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x, amax)
+    x = x.contiguous()
+    st = lib().fp4q_tensor_amax_accumulate(_ptr(x), x.shape[0], x.shape[1], rot, _ptr(amax), _stream(stream))
+    _check(st, "fp4q_tensor_amax_accumulate")
     return amax
 
 

@@ -74,17 +74,21 @@ void set_global(int gmode, float* gscale, const float** gsrc, float** gdst)
     *gdst = gmode == FP4Q_GLOBAL_FROM_AMAX ? gscale + 1 : nullptr;
 }
 
-// amax(|y|) of the tensor into *dst (fp32 bits, via atomicMax on a zeroed slot).
-cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStream_t s)
+// *dst = max(*dst, amax(|y|)) (fp32 bits, atomicMax: non-negative floats order
+// as integers); with `zero` the slot is cleared first.
+cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStream_t s, bool zero = true)
 {
-    cudaError_t e = cudaMemsetAsync(dst, 0, sizeof(float), s);
-    if (e != cudaSuccess || n == 0) return e;
+    if (zero) {
+        cudaError_t e = cudaMemsetAsync(dst, 0, sizeof(float), s);
+        if (e != cudaSuccess) return e;
+    }
+    if (n == 0) return cudaSuccess;
     AmaxParams ap{};
     ap.x = static_cast<const uint16_t*>(x);
     ap.n = n;
     ap.amax_bits = reinterpret_cast<unsigned int*>(dst);
     rotation_constants(rot, &ap.c_hi, &ap.c_lo);
-    return launch_amax(rot, ap, s);
+    return launch_amax(rot, ap, s, !zero);
 }
 
 // ---- fixed scratch of fp4q_block_mse_noalloc
@@ -234,6 +238,16 @@ int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* 
     if (!amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
     if (!aligned(amax, 4) || (n > 0 && !aligned(x, 32))) return FP4Q_ERR_ALIGN;
     return cuda_status(enqueue_amax(x, n, rot, amax, as_stream(stream)));
+}
+
+int fp4q_tensor_amax_accumulate(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, FP4Q_SCALE_E8M0, 8, rot, &n);
+    if (st) return st;
+    if (!amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
+    if (!aligned(amax, 4) || (n > 0 && !aligned(x, 32))) return FP4Q_ERR_ALIGN;
+    return cuda_status(enqueue_amax(x, n, rot, amax, as_stream(stream), false));
 }
 
 int fp4q_global_scale(const float* amax, float* gscale, void* stream)

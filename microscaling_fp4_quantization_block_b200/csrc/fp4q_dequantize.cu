@@ -13,15 +13,14 @@ cudaError_t run_dequantize(const DequantParams& p, cudaStream_t s)
         auto kern = dequantize_il_kernel<B, K, F32>;
         const int64_t tiles = (p.n + kDqTile - 1) / kDqTile;
         const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
-        kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+        return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
     } else {
         auto kern = dequantize_kernel<B, K, F32>;
         const int64_t tile_elems = 32 * DPL;  // 32 lanes x 128 elements
         const int64_t tiles = (p.n + tile_elems - 1) / tile_elems;
         const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
-        kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+        return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
     }
-    return cudaGetLastError();
 }
 
 template <int B, int K>
@@ -38,8 +37,7 @@ cudaError_t run_mse(const MseParams& p, int* grid_out, cudaStream_t s)
     if (need > partial_slots(p.n)) need = partial_slots(p.n);
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
     *grid_out = grid;
-    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
 }
 
 #define FP4Q_BK_SWITCH(B, K, CALL)                                                   \

@@ -88,6 +88,13 @@ __device__ __forceinline__ void stg64(void* p, uint32_t a, uint32_t b)
     asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on have completed and their memory is
+// visible (a no-op for a plain launch), then let the next grid in the stream
+// be scheduled as this one's CTAs retire.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- async copies into shared memory
 // 16-byte global -> shared copy (L2 only, no L1); src_bytes 0 writes zeros and
 // reads nothing.  Completion is tracked per thread with commit / wait groups.

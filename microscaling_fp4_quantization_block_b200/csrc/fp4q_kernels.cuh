@@ -575,6 +575,8 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
 template <int FMT, int B, int K, bool MSE>
 __global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantParams p)
 {
+    pdl_wait();
+    pdl_release();
     extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
@@ -624,6 +626,8 @@ struct AmaxParams {
 template <int K>
 __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
 {
+    pdl_wait();
+    pdl_release();
     extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
@@ -728,6 +732,8 @@ __device__ __forceinline__ void fetch_scale_bytes(const uint8_t* __restrict__ sc
 template <int B, int K, bool F32OUT>
 __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
 {
+    pdl_wait();
+    pdl_release();
     constexpr int NSB = DeqScales<B>::NSB;
     constexpr int EPB = B <= DPL ? B : DPL;                       // elements of a block in a lane
     using R = Ring<64, 1>;                                        // 64 code bytes per lane per tile
@@ -891,6 +897,8 @@ template <int B, int K, bool F32OUT>
 __global__ void __launch_bounds__(kThreads) dequantize_il_kernel(DequantParams p)
 {
     static_assert(K == 0 || K == kDqChunk, "interleaved chunks hold rotation runs of at most 16");
+    pdl_wait();
+    pdl_release();
     using D = DqStage<B>;
     extern __shared__ __align__(128) uint8_t smem_ring[];
     __shared__ float tab[256];                                   // block scale by code
@@ -1047,6 +1055,8 @@ __device__ __forceinline__ void load_unit_codes(const uint8_t* __restrict__ code
 template <int B, int K>
 __global__ void __launch_bounds__(kThreads) block_mse_kernel(MseParams p)
 {
+    pdl_wait();
+    pdl_release();
     using S = UnitShape<B, K>;
     constexpr int NB = S::NB, BE = S::BE, LPB = S::LPB;
     extern __shared__ __align__(128) uint8_t smem_ring[];

@@ -29,9 +29,32 @@ cudaError_t launch_quantize(int fmt, int B, int K, bool mse, const QuantParams& 
 cudaError_t launch_quantize_e8m0(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 cudaError_t launch_quantize_ue4m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 cudaError_t launch_quantize_ue5m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
-cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s);
+// pdl: launch with programmatic dependent launch (never right after the memset
+// that zeroes the maximum's slot, which must complete first).
+cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_dequantize(int B, int K, bool f32out, const DequantParams& p, cudaStream_t s);
 cudaError_t launch_block_mse(int B, int K, const MseParams& p, int* grid_out, cudaStream_t s);
+
+// Launch of a streaming kernel with programmatic dependent launch allowed: the
+// grid may be scheduled while the stream's previous kernel drains, and every
+// such kernel executes griddepcontrol.wait (pdl_wait) before it touches global
+// memory, so it observes everything the stream ordered before it exactly as
+// with a plain launch; only launch and scheduling latency overlap.
+template <typename P>
+inline cudaError_t launch_pdl(void (*kernel)(P), int grid, int threads, int smem, cudaStream_t s, const P& p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
 
 // Upper bound on the CTAs of any kernel that writes per-CTA partials, and the
 // number of partial slots (4 doubles each) a workspace must hold for n elements.

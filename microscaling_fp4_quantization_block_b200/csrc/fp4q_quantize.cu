@@ -57,23 +57,24 @@ cudaError_t launch_quantize(int fmt, int B, int K, bool mse, const QuantParams& 
 namespace {
 
 template <int K>
-cudaError_t run_amax(const AmaxParams& p, cudaStream_t s)
+cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
     auto kern = amax_kernel<K>;
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));
+    if (pdl) return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
     kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s)
+cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl)
 {
     switch (K) {
-    case 0: return run_amax<0>(p, s);
-    case 16: return run_amax<16>(p, s);
-    case 32: return run_amax<32>(p, s);
-    case 128: return run_amax<128>(p, s);
+    case 0: return run_amax<0>(p, s, pdl);
+    case 16: return run_amax<16>(p, s, pdl);
+    case 32: return run_amax<32>(p, s, pdl);
+    case 128: return run_amax<128>(p, s, pdl);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -16,8 +16,7 @@ cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
     if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
     if (grid_out) *grid_out = grid;
-    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
 }
 
 template <int FMT, int B, int K>

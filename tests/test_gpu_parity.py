@@ -295,6 +295,22 @@ def test_mse_workspace_counter_is_left_zero_and_reusable(fq):
         assert np.allclose(t_shared.cpu().numpy(), u_shared.cpu().numpy(), rtol=1e-6, atol=0)
 
 
+@pytest.mark.parametrize("rot", [0, 32])
+def test_amax_accumulate_over_shards(fq, rot):
+    """Row shards folded into one slot give the whole tensor's maximum; a larger
+    value already in the slot is kept."""
+    x, _ = workloads.student_t_outliers_bf16(768, 1024, seed=41 + rot)
+    xd = x.cuda()
+    whole = fq.fp4q_tensor_amax(xd, rot)
+    acc = torch.zeros(1, dtype=torch.float32, device="cuda")
+    for r0 in range(0, 768, 256):
+        fq.fp4q_tensor_amax_accumulate(xd[r0:r0 + 256], acc, rot)
+    big = torch.full((1,), 1e30, dtype=torch.float32, device="cuda")
+    fq.fp4q_tensor_amax_accumulate(xd, big, rot)
+    torch.cuda.synchronize()
+    assert acc.item() == whole.item() and big.item() == np.float32(1e30)
+
+
 FUSED_CASES = [(E8, 32, 0, NONE), (U4, 16, 0, COMP), (U4, 16, 0, NONE), (U4, 8, 0, NONE), (E8, 256, 0, NONE),
                (U5, 64, 0, NONE), (E8, 32, 32, NONE), (U4, 16, 128, COMP), (U4, 256, 16, NONE),
                (E8, 8, 128, NONE)]
