@@ -134,6 +134,27 @@ __device__ __forceinline__ uint32_t e2m1_pack8(float v0, float v1, float v2, flo
     return r;
 }
 
+// Codes of 8 values -> code word, plus each code byte decoded back to an
+// f16x2 pair (h[j] = grid values of elements 2j, 2j+1) for the MSE.
+__device__ __forceinline__ uint32_t e2m1_pack8_dec(float v0, float v1, float v2, float v3, float v4, float v5,
+                                                   float v6, float v7, uint32_t (&h)[4])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t}"
+        : "=r"(r), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return r;
+}
+
 // Two nibbles (one code byte, low nibble first) -> two exact fp32 values.
 __device__ __forceinline__ void e2m1_unpack2(uint32_t byte, float& lo, float& hi)
 {

@@ -322,6 +322,17 @@ __device__ __forceinline__ uint32_t pack_pairs(f32x2 p0, f32x2 p1, f32x2 p2, f32
     return e2m1_pack8(a0, b0, a1, b1, a2, b2, a3, b3);
 }
 
+// E2M1 codes of 4 pairs -> code word, and the grid values decoded back (f16x2 per pair).
+__device__ __forceinline__ uint32_t pack_pairs_dec(f32x2 p0, f32x2 p1, f32x2 p2, f32x2 p3, uint32_t (&h)[4])
+{
+    float a0, b0, a1, b1, a2, b2, a3, b3;
+    upk(p0, a0, b0);
+    upk(p1, a1, b1);
+    upk(p2, a2, b2);
+    upk(p3, a3, b3);
+    return e2m1_pack8_dec(a0, b0, a1, b1, a2, b2, a3, b3, h);
+}
+
 // Codes of 4 pairs with correctly rounded quotients v / s (s != 0) by
 // division: the fallback for scales outside the range the remainder
 // correction serves (extreme per-tensor scales), kept out of line.
@@ -461,60 +472,72 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     uint32_t code[NB];
     const bool exact = unit_scales<FMT, NB>(m, kc, tab, code, sc, rm);
 
+    // ---- codes, one 8-element word at a time; each word's code bytes are also
+    // decoded straight back for the MSE, whose squared errors are taken right
+    // away (three-term split of "Finer is better?": v_i = fp32(decode(code_i) * S))
     uint32_t cw[EPT / 8];
-    if constexpr (FMT == kE8M0) {
-        // S is a power of two: y * (1/S) is the quotient itself.
+    f32x2 bsum[NB];
 #pragma unroll
-        for (int k = 0; k < EPT / 8; ++k) {
-            const f32x2 r = pk(rm[(8 * k) / BE], rm[(8 * k) / BE]);
-            cw[k] = pack_pairs(mul2(v[4 * k], r), mul2(v[4 * k + 1], r), mul2(v[4 * k + 2], r),
-                               mul2(v[4 * k + 3], r));
-        }
-    } else {
-        if (exact) {
-            // correctly rounded quotients y / S (remainder correction), then the
-            // hardware E2M1 rounding (nearest, ties to the even code, saturating)
+    for (int bi = 0; bi < NB; ++bi) bsum[bi] = pk(0.0f, 0.0f);
+    const f32x2 nz2 = pk(nz, nz);                // -0: fma(g, S, -0) is the rounded product fp32(g S)
+    bool anyzero = false;
+    if constexpr (FMT != kE8M0) {
 #pragma unroll
-            for (int k = 0; k < EPT / 8; ++k) {
-                const int bi = (8 * k) / BE;
-                const f32x2 R2 = pk(rm[bi], rm[bi]), nS2 = pk(-sc[bi], -sc[bi]);
-                cw[k] = pack_pairs(div2_cr(v[4 * k], R2, nS2), div2_cr(v[4 * k + 1], R2, nS2),
-                                   div2_cr(v[4 * k + 2], R2, nS2), div2_cr(v[4 * k + 3], R2, nS2));
-            }
+        for (int bi = 0; bi < NB; ++bi) anyzero |= sc[bi] == 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < EPT / 8; ++k) {
+        const int bi = (8 * k) / BE;
+        const f32x2* vk = v + 4 * k;
+        uint32_t h[4];
+        if constexpr (FMT == kE8M0) {
+            // S is a power of two: y * (1/S) is the quotient itself.
+            const f32x2 r = pk(rm[bi], rm[bi]);
+            cw[k] = pack_pairs_dec(mul2(vk[0], r), mul2(vk[1], r), mul2(vk[2], r), mul2(vk[3], r), h);
         } else {
-            // extreme scales: correctly rounded divisions
+            if (exact) {
+                // correctly rounded quotients y / S (remainder correction), then the
+                // hardware E2M1 rounding (nearest, ties to the even code, saturating)
+                const f32x2 R2 = pk(rm[bi], rm[bi]), nS2 = pk(-sc[bi], -sc[bi]);
+                cw[k] = pack_pairs_dec(div2_cr(vk[0], R2, nS2), div2_cr(vk[1], R2, nS2), div2_cr(vk[2], R2, nS2),
+                                       div2_cr(vk[3], R2, nS2), h);
+            } else {
+                // extreme scales: correctly rounded divisions
+                cw[k] = sc[bi] != 0.0f ? pack_pairs_div(vk[0], vk[1], vk[2], vk[3], sc[bi]) : 0u;
 #pragma unroll
-            for (int k = 0; k < EPT / 8; ++k) {
-                const float s = sc[(8 * k) / BE];
-                cw[k] = s != 0.0f ? pack_pairs_div(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], s) : 0u;
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t hh;
+                    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(hh) : "r"((cw[k] >> (8 * j)) & 0xffu));
+                    h[j] = hh;
+                }
             }
         }
-        // zero-rounded blocks store plain 0x0 nibbles
+        if constexpr (MSE) {
+            // zero-rounded blocks (S = 0) give v = 0 whatever the decoded bytes
+            const f32x2 s2 = pk(sc[bi], sc[bi]);
 #pragma unroll
-        for (int k = 0; k < EPT / 8; ++k)
-            if (sc[(8 * k) / BE] == 0.0f) cw[k] = 0u;
+            for (int j = 0; j < 4; ++j) {
+                __half2 hh = *reinterpret_cast<__half2*>(&h[j]);
+                const f32x2 g = pk(__low2float(hh), __high2float(hh));
+                const f32x2 d = sub2(vk[j], fma2(g, s2, nz2));     // y - fp32(g S)
+                bsum[bi] = fma2(d, d, bsum[bi]);
+            }
+        }
+    }
+    if constexpr (FMT != kE8M0) {
+        if (anyzero) {
+#pragma unroll
+            for (int k = 0; k < EPT / 8; ++k)
+                if (sc[(8 * k) / BE] == 0.0f) cw[k] = 0u;      // zero-rounded blocks store plain 0x0 nibbles
+        }
     }
 
-    // ---- fused MSE (three-term split of "Finer is better?"): v_i = fp32(decode(code_i) * S)
     if constexpr (MSE) {
-        const f32x2 nz2 = pk(nz, nz);            // -0: fma(g, S, -0) is the rounded product fp32(g S)
         float tot = 0.0f, mx = 0.0f, zr = 0.0f;
 #pragma unroll
         for (int bi = 0; bi < NB; ++bi) {
-            const f32x2 s2 = pk(sc[bi], sc[bi]);
-            f32x2 sum = pk(0.0f, 0.0f);
-#pragma unroll
-            for (int k = bi * BE / 8; k < (bi + 1) * BE / 8; ++k) {
-                f32x2 g[4];
-                decode8(cw[k], g);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const f32x2 d = sub2(v[4 * k + j], fma2(g[j], s2, nz2));     // y - fp32(g S)
-                    sum = fma2(d, d, sum);
-                }
-            }
             float se, so;
-            upk(sum, se, so);
+            upk(bsum[bi], se, so);
             float s = __fadd_rn(se, so);
             if constexpr (S::LPB > 1) s = group_sum<S::LPB>(s);
             const float vmax = block_vmax<FMT>(m[bi], sc[bi], rm[bi], code[bi], exact);
@@ -572,8 +595,11 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     }
 }
 
+// Two CTAs per SM (up to 128 registers) unless the kernel fits three without
+// spilling: measured, spills in the UE and fused variants cost more than the
+// extra warps gain.
 template <int FMT, int B, int K, bool MSE>
-__global__ void __launch_bounds__(kThreads, MSE ? 2 : 3) quantize_kernel(QuantParams p)
+__global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quantize_kernel(QuantParams p)
 {
     pdl_wait();
     pdl_release();
