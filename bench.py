@@ -51,7 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--separate-mse", action="store_true",
-                    help="measure the MSE with its own pass over x (fp4q_quantize + fp4q_block_mse)")
+                    help="measure the MSE with its own pass over x (fp4q_quantize + fp4q_block_mse + fp4q_dequantize)")
+    ap.add_argument("--separate-dequant", action="store_true",
+                    help="dequantize with its own pass over the codes (fp4q_quantize_mse + fp4q_dequantize)")
     return ap.parse_args(argv)
 
 
@@ -115,6 +117,7 @@ def bytes_per_element(block: int):
         "amax": 2.0,
         "quantize": 2.0 + 0.5 + 1.0 / block,
         "quantize_mse": 2.0 + 0.5 + 1.0 / block + 4.0 / block,
+        "quantize_mse_dequantize": 2.0 + 0.5 + 1.0 / block + 4.0 / block + 2.0,
         "dequantize": 0.5 + 1.0 / block + 2.0,
         "block_mse": 2.0 + 0.5 + 1.0 / block + 4.0 / block,
     }
@@ -130,7 +133,7 @@ class Pipeline:
     """
 
 
-    def __init__(self, fq, items, device, stream, separate_mse=False):
+    def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False):
         import torch
         self.fq, self.items, self.device = fq, items, device
         L = fq.lib()
@@ -168,17 +171,24 @@ class Pipeline:
                 seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
                                                             fmt, block, rot, p["bm"], p["terms"], p["ws"],
                                                             b["ws"].numel(), sh)))
-            else:
+            elif separate_dequant:
                 seq.append(("quantize_mse", L.fp4q_quantize_mse,
                             (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], gq, p["bm"],
                              p["terms"], p["ws"], b["ws"].numel(), sh)))
-            seq.append(("dequantize", L.fp4q_dequantize, (p["codes"], p["scales"], g, rows, cols, fmt, block, 0,
-                                                          0, p["deq"], sh)))
+            else:
+                # quantize, the MSE split and the dequantized bf16 tensor in one pass over x
+                seq.append(("quantize_mse_dequantize", L.fp4q_quantize_mse_dequantize,
+                            (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], gq, p["deq"],
+                             p["bm"], p["terms"], p["ws"], b["ws"].numel(), sh)))
+            if separate_mse or separate_dequant:
+                seq.append(("dequantize", L.fp4q_dequantize, (p["codes"], p["scales"], g, rows, cols, fmt, block, 0,
+                                                              0, p["deq"], sh)))
             self.calls.append(seq)
         self.elements = sum(x.numel() for _, x, *_ in items)
-        # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel), [block MSE], dequantize
-        self.launches_per_step = sum(2 + (1 if gm == COMP else 0) + (1 if separate_mse else 0)
-                                     for *_, gm in items)
+        # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel, + dequantized output),
+        # [block MSE], [dequantize]
+        self.launches_per_step = sum(1 + (1 if gm == COMP else 0) + (2 if separate_mse else 0)
+                                     + (1 if separate_dequant and not separate_mse else 0) for *_, gm in items)
         self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
 
     def step(self, stream, ev=None):
@@ -406,7 +416,8 @@ def main(argv=None):
     items = build_workload(args.workload, device, rank, args)
     stream = torch.cuda.Stream(device)
     stream.wait_stream(torch.cuda.current_stream())
-    pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse)
+    pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse,
+                    separate_dequant=args.separate_dequant)
     in_l2 = sum(x.numel() * 2 for _, x, *_ in items) < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
 

@@ -196,6 +196,20 @@ FP4Q_API int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fm
                                float* block_mse, double* terms, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/*
+ * fp4q_quantize_mse_dequantize -- fp4q_quantize_mse that also writes the
+ * dequantized tensor: y (bf16 [rows][cols], 32-byte aligned) receives exactly
+ * what fp4q_dequantize(codes, scales, G, ..., rot = 0, FP4Q_OUT_BF16) would
+ * write (values in the quantized, i.e. rotated, domain), computed from the
+ * values the MSE already forms, so the codes are not read back ("Diagnosing
+ * FP4 inference", Methodology: quantized on the fly, then dequantized for the
+ * compute).  Other arguments, outputs and errors as fp4q_quantize_mse.
+ */
+FP4Q_API int fp4q_quantize_mse_dequantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                          int gmode, uint8_t* codes, uint8_t* scales, float* gscale, void* y,
+                                          float* block_mse, double* terms, void* workspace, size_t ws_bytes,
+                                          void* stream);
+
 /* Bytes of device workspace fp4q_block_mse and fp4q_quantize_mse need for this
  * shape (host only; at most 128 KiB + 16): the completion counter and the
  * per-CTA partials. */

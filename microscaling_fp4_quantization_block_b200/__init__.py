@@ -52,6 +52,7 @@ def _load() -> ctypes.CDLL:
         "fp4q_block_mse_workspace_size": (SZ, [I64, I64, I]),
         "fp4q_block_mse_noalloc": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P]),
         "fp4q_quantize_mse": (I, [P, I64, I64, I, I, I, I, P, P, P, P, P, P, SZ, P]),
+        "fp4q_quantize_mse_dequantize": (I, [P, I64, I64, I, I, I, I, P, P, P, P, P, P, P, SZ, P]),
         "fp4q_e2m1_encode_f32": (I, [P, I64, P, P]),
         "fp4q_scale_encode_f32": (I, [P, I64, I, P, P]),
         "fp4q_status_string": (ctypes.c_char_p, [I]),
@@ -279,6 +280,46 @@ def fp4q_quantize_mse(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="non
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "fp4q_quantize_mse")
     return codes, scales, gscale, block_mse, terms
+
+
+def fp4q_quantize_mse_dequantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
+                                 codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                                 gscale: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                                 block_mse: Optional[torch.Tensor] = None, want_block_mse: bool = True,
+                                 terms: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                                 stream=None):
+    """Quantize, measure the MSE and write the dequantized bf16 tensor in one pass:
+    (codes, scales, gscale, y, block_mse, terms)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    fmt, gmode = _fmt(fmt), _gmode(gmode)
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // block if block else 0), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode == FP4Q_GLOBAL_FROM_AMAX:
+        raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
+    if gscale is None and gmode != FP4Q_GLOBAL_NONE:
+        gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    if y is None:
+        y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    if block_mse is None and want_block_mse:
+        block_mse = torch.empty((rows, cols // block if block else 0), dtype=torch.float32, device=dev)
+    if terms is None:
+        terms = torch.empty((4,), dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.zeros((fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
+                                device=dev)
+    _need_cuda(codes, scales, gscale, y, block_mse, terms, workspace)
+    st = lib().fp4q_quantize_mse_dequantize(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(codes), _ptr(scales),
+                                            _ptr(gscale), _ptr(y), _ptr(block_mse), _ptr(terms), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "fp4q_quantize_mse_dequantize")
+    return codes, scales, gscale, y, block_mse, terms
 
 
 def fp4q_e2m1_encode_f32(r: torch.Tensor, packed: Optional[torch.Tensor] = None,

@@ -120,6 +120,59 @@ int noalloc_partials_for_current_device(double** out)
     return FP4Q_OK;
 }
 
+// fp4q_quantize_mse, with the dequantized values written to y (bf16) when y is set.
+int quantize_mse_impl(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                      uint8_t* codes, uint8_t* scales, float* gscale, void* y, float* block_mse, double* terms,
+                      void* workspace, size_t ws_bytes, void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
+    if (gmode != FP4Q_GLOBAL_NONE) {
+        if (!gscale) return FP4Q_ERR_NULL;
+        if (!aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
+    }
+    if (!terms || !workspace) return FP4Q_ERR_NULL;
+    if (!aligned(terms, 8) || !aligned(workspace, 8)) return FP4Q_ERR_ALIGN;
+    if (n > 0) {
+        if (!x || !codes || !scales) return FP4Q_ERR_NULL;
+        if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)) return FP4Q_ERR_ALIGN;
+        if (y && !aligned(y, 32)) return FP4Q_ERR_ALIGN;
+    }
+    if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
+    if (ws_bytes < fp4q_block_mse_workspace_size(rows, cols, block)) return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    if (gmode == FP4Q_GLOBAL_COMPUTE) {
+        cudaError_t e = enqueue_amax(x, n, rot, gscale, s);
+        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+        global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
+        if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    if (n == 0) {
+        if (gmode == FP4Q_GLOBAL_FROM_AMAX) {
+            global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale + 1);
+            if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+        }
+        return cuda_status(cudaMemsetAsync(terms, 0, 4 * sizeof(double), s));
+    }
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.n = n;
+    p.codes = codes;
+    p.scales = scales;
+    set_global(gmode, gscale, &p.gsrc, &p.gdst);
+    p.block_mse = block_mse;
+    p.partials = mse_partials(workspace);
+    p.done = mse_counter(workspace);
+    p.terms = terms;
+    p.y = static_cast<uint16_t*>(y);
+    rotation_constants(rot, &p.c_hi, &p.c_lo);
+    int grid = 0;
+    return cuda_status(launch_quantize(fmt, block, rot, true, p, &grid, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -184,50 +237,17 @@ int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int bl
                       uint8_t* codes, uint8_t* scales, float* gscale, float* block_mse, double* terms,
                       void* workspace, size_t ws_bytes, void* stream)
 {
-    int64_t n = 0;
-    int st = check_shape(rows, cols, fmt, block, rot, &n);
-    if (st) return st;
-    if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
-    if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
-    if (gmode != FP4Q_GLOBAL_NONE) {
-        if (!gscale) return FP4Q_ERR_NULL;
-        if (!aligned(gscale, 4)) return FP4Q_ERR_ALIGN;
-    }
-    if (!terms || !workspace) return FP4Q_ERR_NULL;
-    if (!aligned(terms, 8) || !aligned(workspace, 8)) return FP4Q_ERR_ALIGN;
-    if (n > 0) {
-        if (!x || !codes || !scales) return FP4Q_ERR_NULL;
-        if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(scales, 16)) return FP4Q_ERR_ALIGN;
-    }
-    if (block_mse && !aligned(block_mse, 16)) return FP4Q_ERR_ALIGN;
-    if (ws_bytes < fp4q_block_mse_workspace_size(rows, cols, block)) return FP4Q_ERR_WORKSPACE;
-    cudaStream_t s = as_stream(stream);
-    if (gmode == FP4Q_GLOBAL_COMPUTE) {
-        cudaError_t e = enqueue_amax(x, n, rot, gscale, s);
-        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
-        global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale);
-        if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
-    }
-    if (n == 0) {
-        if (gmode == FP4Q_GLOBAL_FROM_AMAX) {
-            global_scale_kernel<<<1, 1, 0, s>>>(gscale, gscale + 1);
-            if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
-        }
-        return cuda_status(cudaMemsetAsync(terms, 0, 4 * sizeof(double), s));
-    }
-    QuantParams p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.n = n;
-    p.codes = codes;
-    p.scales = scales;
-    set_global(gmode, gscale, &p.gsrc, &p.gdst);
-    p.block_mse = block_mse;
-    p.partials = mse_partials(workspace);
-    p.done = mse_counter(workspace);
-    p.terms = terms;
-    rotation_constants(rot, &p.c_hi, &p.c_lo);
-    int grid = 0;
-    return cuda_status(launch_quantize(fmt, block, rot, true, p, &grid, s));
+    return quantize_mse_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, nullptr, block_mse,
+                             terms, workspace, ws_bytes, stream);
+}
+
+int fp4q_quantize_mse_dequantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                 int gmode, uint8_t* codes, uint8_t* scales, float* gscale, void* y,
+                                 float* block_mse, double* terms, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (rows > 0 && cols > 0 && !y) return FP4Q_ERR_NULL;
+    return quantize_mse_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, y, block_mse, terms,
+                             workspace, ws_bytes, stream);
 }
 
 int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)

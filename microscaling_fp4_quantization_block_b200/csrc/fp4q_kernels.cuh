@@ -451,9 +451,10 @@ struct QuantParams {
     unsigned int* done;    // fused MSE: completion counter (0 at launch, left 0)
     double* terms;         // fused MSE: the four tensor terms
     float* gdst;           // G from the tensor maximum: *gsrc is that maximum, G is written here
+    uint16_t* y;           // fused MSE with dequantized output: n bf16 values
 };
 
-template <int FMT, int B, int K, bool MSE>
+template <int FMT, int B, int K, bool MSE, bool DQ>
 __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
                                               int lane, const ScaleConsts& kc, const float2* tab, float nz,
                                               double (&acc)[3])
@@ -515,20 +516,49 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
         if constexpr (MSE) {
             // zero-rounded blocks (S = 0) give v = 0 whatever the decoded bytes
             const f32x2 s2 = pk(sc[bi], sc[bi]);
+            uint32_t yw[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 __half2 hh = *reinterpret_cast<__half2*>(&h[j]);
                 const f32x2 g = pk(__low2float(hh), __high2float(hh));
-                const f32x2 d = sub2(vk[j], fma2(g, s2, nz2));     // y - fp32(g S)
+                const f32x2 vq = fma2(g, s2, nz2);                   // v = fp32(g S)
+                const f32x2 d = sub2(vk[j], vq);                     // y - v
                 bsum[bi] = fma2(d, d, bsum[bi]);
+                if constexpr (DQ) {
+                    float a, b;
+                    upk(vq, a, b);
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+                    yw[j] = *reinterpret_cast<uint32_t*>(&hb);
+                }
+            }
+            if constexpr (DQ) {
+                // the dequantized values of this word, as fp4q_dequantize writes them
+                const int64_t ew = u * EPT + 8 * k;
+                if (ew + 8 <= p.n) {
+                    stg128(p.y + ew, yw[0], yw[1], yw[2], yw[3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (ew + 2 * j < p.n) p.y[ew + 2 * j] = (uint16_t)(yw[j] & 0xffffu);
+                        if (ew + 2 * j + 1 < p.n) p.y[ew + 2 * j + 1] = (uint16_t)(yw[j] >> 16);
+                    }
+                }
             }
         }
     }
     if constexpr (FMT != kE8M0) {
         if (anyzero) {
 #pragma unroll
-            for (int k = 0; k < EPT / 8; ++k)
-                if (sc[(8 * k) / BE] == 0.0f) cw[k] = 0u;      // zero-rounded blocks store plain 0x0 nibbles
+            for (int k = 0; k < EPT / 8; ++k) {
+                if (sc[(8 * k) / BE] == 0.0f) {
+                    cw[k] = 0u;                                // zero-rounded blocks store plain 0x0 nibbles
+                    if constexpr (DQ) {                        // ... which dequantize to +0
+                        const int64_t ew = u * EPT + 8 * k;
+                        for (int j = 0; j < 8; ++j)
+                            if (ew + j < p.n) p.y[ew + j] = 0u;
+                    }
+                }
+            }
         }
     }
 
@@ -598,7 +628,7 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
 // Two CTAs per SM (up to 128 registers) unless the kernel fits three without
 // spilling: measured, spills in the UE and fused variants cost more than the
 // extra warps gain.
-template <int FMT, int B, int K, bool MSE>
+template <int FMT, int B, int K, bool MSE, bool DQ = false>
 __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quantize_kernel(QuantParams p)
 {
     pdl_wait();
@@ -633,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quant
                  [&](int64_t t, int s) {
                      uint32_t w[EPT / 2];
                      ring.read(s, 0, w);
-                     quantize_unit<FMT, B, K, MSE>(p, t * 32 + lane, w, lane, kc, tab, nz, acc);
+                     quantize_unit<FMT, B, K, MSE, DQ>(p, t * 32 + lane, w, lane, kc, tab, nz, acc);
                  });
     if constexpr (MSE) {
         cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);

@@ -8,10 +8,10 @@
 namespace fp4q {
 namespace detail {
 
-template <int FMT, int B, int K, bool MSE>
+template <int FMT, int B, int K, bool MSE, bool DQ = false>
 cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
 {
-    auto kern = quantize_kernel<FMT, B, K, MSE>;
+    auto kern = quantize_kernel<FMT, B, K, MSE, DQ>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
@@ -22,7 +22,8 @@ cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
 template <int FMT, int B, int K>
 cudaError_t by_mse(bool mse, const QuantParams& p, int* g, cudaStream_t s)
 {
-    return mse ? run_quantize<FMT, B, K, true>(p, g, s) : run_quantize<FMT, B, K, false>(p, g, s);
+    if (!mse) return run_quantize<FMT, B, K, false>(p, g, s);
+    return p.y ? run_quantize<FMT, B, K, true, true>(p, g, s) : run_quantize<FMT, B, K, true>(p, g, s);
 }
 
 template <int FMT, int B>

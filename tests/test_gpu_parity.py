@@ -335,6 +335,39 @@ def test_fused_quantize_mse_matches_separate_calls(fq, fmt, block, rot, gmode):
     assert_mse_close(bm.cpu().numpy(), terms.cpu().numpy(), o_bm, o_terms, 2e-6 if rot == 0 else 1e-5)
 
 
+@pytest.mark.parametrize("fmt,block,rot,gmode", FUSED_CASES)
+def test_fused_dequantized_output_equals_dequantize(fq, fmt, block, rot, gmode):
+    """fp4q_quantize_mse_dequantize: codes, scales, G and MSE as fp4q_quantize_mse,
+    and y bit for bit what fp4q_dequantize (bf16, quantized domain) writes."""
+    x, _ = workloads.student_t_outliers_bf16(333, 1024, seed=7 * block + rot)
+    xd = x.cuda()
+    c1, s1, g1, bm1, t1 = fq.fp4q_quantize_mse(xd, fmt, block, rot, gmode)
+    c2, s2, g2, y, bm2, t2 = fq.fp4q_quantize_mse_dequantize(xd, fmt, block, rot, gmode)
+    ref = fq.fp4q_dequantize(c2, s2, g2 if fmt != E8 else None, 333, 1024, fmt, block, 0, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2) and torch.equal(bm1, bm2)
+    assert t1.cpu().numpy().tobytes() == t2.cpu().numpy().tobytes()
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+
+
+def test_fused_dequantized_output_zero_blocks_and_signed_zeros(fq):
+    """Zero-rounded blocks give +0, a negative value that rounds to zero -0, and a
+    ragged tail; all as fp4q_dequantize."""
+    for fmt, block, gmode, gval in [(U4, 16, GIVEN, 1.0), (U4, 8, NONE, None), (E8, 32, NONE, None)]:
+        cols = 4096 + block                      # 9 rows: the last unit is partial for b8 and b16
+        x = workloads.gaussian_bf16(9, cols, 0.02, seed=12)
+        x[0, :64] = 0.0
+        x[1, :16] = 1e-7
+        x[1, 16:32] = -1e-7
+        x[2, 5] = -0.0
+        xd = x.cuda()
+        gs = torch.tensor([gval], dtype=torch.float32, device="cuda") if gval is not None else None
+        c, s, g, y, bm, t = fq.fp4q_quantize_mse_dequantize(xd, fmt, block, 0, gmode, gscale=gs)
+        ref = fq.fp4q_dequantize(c, s, g if fmt != E8 else None, 9, cols, fmt, block, 0, torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), fmt
+
+
 def test_fused_quantize_mse_full_gaussian(fq):
     x = workloads.gaussian_bf16(2048, 3584, 0.005, seed=21)
     xb = bf16_bits(x)
