@@ -477,6 +477,7 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     // decoded straight back for the MSE, whose squared errors are taken right
     // away (three-term split of "Finer is better?": v_i = fp32(decode(code_i) * S))
     uint32_t cw[EPT / 8];
+    uint32_t ypend[4];                           // bf16 words of the previous (even) word, stored in pairs
     f32x2 bsum[NB];
 #pragma unroll
     for (int bi = 0; bi < NB; ++bi) bsum[bi] = pk(0.0f, 0.0f);
@@ -532,10 +533,16 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
                 }
             }
             if constexpr (DQ) {
-                // the dequantized values of this word, as fp4q_dequantize writes them
+                // the dequantized values of this word, as fp4q_dequantize writes them;
+                // two words (32 bytes) per store
                 const int64_t ew = u * EPT + 8 * k;
-                if (ew + 8 <= p.n) {
-                    stg128(p.y + ew, yw[0], yw[1], yw[2], yw[3]);
+                if (u * EPT + EPT <= p.n) {
+                    if ((k & 1) == 0) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) ypend[j] = yw[j];
+                    } else {
+                        stg256(p.y + ew - 8, ypend[0], ypend[1], ypend[2], ypend[3], yw[0], yw[1], yw[2], yw[3]);
+                    }
                 } else {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
