@@ -70,6 +70,10 @@ def lib() -> ctypes.CDLL:
             "orc_quantize_f32": (I, [P, I64, I64, I, I, I, I, P, P, P]),
             "orc_quantize_bf16": (I, [P, I64, I64, I, I, I, I, P, P, P]),
             "orc_dequantize": (I, [P, P, F, I64, I64, I, I, I, P]),
+            "orc_quantize_search_f32": (I, [P, I64, I64, I, I, I, I, I, I, P, P, P]),
+            "orc_quantize_search_bf16": (I, [P, I64, I64, I, I, I, I, I, I, P, P, P]),
+            "orc_quantize_with_scales_f32": (I, [P, I64, I64, I, I, I, P, F, P]),
+            "orc_quantize_with_scales_bf16": (I, [P, I64, I64, I, I, I, P, F, P]),
             "orc_block_mse_f32": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
             "orc_block_mse_bf16": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
         }
@@ -204,6 +208,42 @@ def quantize(x, fmt: int, block: int, rot: int = 0, gmode: int = G_NONE, gscale:
     _check(fn(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(g), _ptr(codes), _ptr(scales)),
            "quantize")
     return codes, scales, float(g[0])
+
+
+def quantize_search(x, fmt: int, block: int, rot: int = 0, gmode: int = G_NONE, gscale: float = 1.0,
+                    below: int = 1, above: int = 1):
+    """Quantize with MSE-optimised block scales: per block, the max-rule code and
+    the codes up to `above` above and `below` below it are tried (in that order)
+    and the one of least squared error is kept (ties keep the earlier one).
+
+    Returns ``(codes, scales, G)`` like :func:`quantize`.
+    """
+    x = np.ascontiguousarray(x)
+    if x.ndim != 2:
+        raise ValueError("expected a 2-D array")
+    if x.dtype not in (np.uint16, np.float32):
+        raise TypeError("x must be float32 values or uint16 bf16 bit patterns")
+    rows, cols = x.shape
+    codes = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // block if block else 0), np.uint8)
+    g = np.array([gscale], np.float32)
+    fn = lib().orc_quantize_search_bf16 if x.dtype == np.uint16 else lib().orc_quantize_search_f32
+    _check(fn(_ptr(x), rows, cols, fmt, block, rot, gmode, below, above, _ptr(g), _ptr(codes), _ptr(scales)),
+           "quantize_search")
+    return codes, scales, float(g[0])
+
+
+def quantize_with_scales(x, scales, G: float, fmt: int, block: int, rot: int = 0) -> np.ndarray:
+    """Codes of x for given scale bytes (each block quantized with its own S)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype not in (np.uint16, np.float32):
+        raise TypeError("x must be float32 values or uint16 bf16 bit patterns")
+    rows, cols = x.shape
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    codes = np.empty((rows, cols // 2), np.uint8)
+    fn = lib().orc_quantize_with_scales_bf16 if x.dtype == np.uint16 else lib().orc_quantize_with_scales_f32
+    _check(fn(_ptr(x), rows, cols, fmt, block, rot, _ptr(scales), G, _ptr(codes)), "quantize_with_scales")
+    return codes
 
 
 def dequantize(codes, scales, G: float, rows: int, cols: int, fmt: int, block: int,

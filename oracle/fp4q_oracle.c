@@ -383,6 +383,130 @@ int orc_quantize_f32(const float* x, int64_t rows, int64_t cols, int fmt, int bl
     return ORC_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* MSE-optimised block scales ([B] s3, MR-GPTQ item 2, "MSE-optimised grids": */
+/* each block's scale is chosen to minimise its squared reconstruction error  */
+/* instead of by the max rule).  The pages give no search procedure; the     */
+/* reading taken here: the candidates are the max-rule code s0 and its        */
+/* neighbours in code order, tried as s0, s0+1 .. s0+above, s0-1 .. s0-below */
+/* (codes outside the format's finite range are skipped); a candidate         */
+/* replaces the best so far only when its error is strictly smaller, so ties  */
+/* keep the earlier one and the max rule wins any tie.  The error of a scale  */
+/* S is sum_i (y_i - v_i)^2 in fp64 with v_i = fp32(decode(E2M1(y_i / S)) S), */
+/* and v_i = 0 when S = 0 (a zero-rounded block).                             */
+
+static int last_finite_code(int fmt)
+{
+    if (fmt == ORC_E8M0) return 0xfe;
+    if (fmt == ORC_UE4M3) return 0x7e;
+    return 0xfe;
+}
+
+static double block_sq_error(const float* y, int block, float S)
+{
+    double sum = 0.0;
+    for (int i = 0; i < block; ++i) {
+        float v = 0.0f;
+        if (S != 0.0f) v = (float)((double)orc_e2m1_decode(orc_e2m1_encode(y[i] / S)) * (double)S);
+        double d = (double)y[i] - (double)v;
+        sum += d * d;
+    }
+    return sum;
+}
+
+int orc_quantize_search_f32(const float* x, int64_t rows, int64_t cols, int fmt, int block,
+                            int rot, int gmode, int below, int above, float* gscale,
+                            uint8_t* codes, uint8_t* scales)
+{
+    if (below < 0 || below > 16 || above < 0 || above > 16) return ORC_EARG;
+    /* the max rule first: its scales are the search's starting codes */
+    int st = orc_quantize_f32(x, rows, cols, fmt, block, rot, gmode, gscale, codes, scales);
+    if (st) return st;
+    const int64_t n = rows * cols;
+    float* y = domain_values(x, n, rot);
+    if (!y) return ORC_ENOMEM;
+    const float G = gmode != ORC_G_NONE ? *gscale : 1.0f;
+    const int last = last_finite_code(fmt);
+
+    memset(codes, 0, (size_t)(n / 2));
+    for (int64_t b0 = 0, bi = 0; b0 < n; b0 += block, ++bi) {
+        const int s0 = scales[bi];
+        int best = s0;
+        double best_err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)s0, G));
+        for (int j = 1; j <= above + below; ++j) {
+            const int c = j <= above ? s0 + j : s0 - (j - above);
+            if (c < 0 || c > last) continue;
+            double err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)c, G));
+            if (err < best_err) {
+                best = c;
+                best_err = err;
+            }
+        }
+        scales[bi] = (uint8_t)best;
+        const float S = scale_of_code(fmt, (uint8_t)best, G);
+        for (int i = 0; i < block; ++i) {
+            uint8_t nib = 0u;
+            if (S != 0.0f) nib = orc_e2m1_encode(y[b0 + i] / S);
+            int64_t e = b0 + i;
+            codes[e >> 1] |= (uint8_t)(nib << ((e & 1) ? 4 : 0));
+        }
+    }
+    free(y);
+    return ORC_OK;
+}
+
+int orc_quantize_search_bf16(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int block,
+                             int rot, int gmode, int below, int above, float* gscale,
+                             uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || cols < 0) return ORC_ESHAPE;
+    const int64_t n = rows * cols;
+    float* xf = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    if (!xf) return ORC_ENOMEM;
+    orc_bf16_to_f32_array(x, n, xf);
+    int st = orc_quantize_search_f32(xf, rows, cols, fmt, block, rot, gmode, below, above, gscale,
+                                     codes, scales);
+    free(xf);
+    return st;
+}
+
+/* Codes for given scale bytes: every block quantized with S = decode(scale)
+ * (times G for the UE formats) exactly as the max rule's blocks are. */
+int orc_quantize_with_scales_f32(const float* x, int64_t rows, int64_t cols, int fmt, int block,
+                                 int rot, const uint8_t* scales, float G, uint8_t* codes)
+{
+    int st = check_layout(rows, cols, fmt, block, rot);
+    if (st) return st;
+    const int64_t n = rows * cols;
+    float* y = domain_values(x, n, rot);
+    if (!y) return ORC_ENOMEM;
+    memset(codes, 0, (size_t)(n / 2));
+    for (int64_t b0 = 0, bi = 0; b0 < n; b0 += block, ++bi) {
+        const float S = scale_of_code(fmt, scales[bi], G);
+        for (int i = 0; i < block; ++i) {
+            uint8_t nib = 0u;
+            if (S != 0.0f) nib = orc_e2m1_encode(y[b0 + i] / S);
+            int64_t e = b0 + i;
+            codes[e >> 1] |= (uint8_t)(nib << ((e & 1) ? 4 : 0));
+        }
+    }
+    free(y);
+    return ORC_OK;
+}
+
+int orc_quantize_with_scales_bf16(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int block,
+                                  int rot, const uint8_t* scales, float G, uint8_t* codes)
+{
+    if (rows < 0 || cols < 0) return ORC_ESHAPE;
+    const int64_t n = rows * cols;
+    float* xf = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    if (!xf) return ORC_ENOMEM;
+    orc_bf16_to_f32_array(x, n, xf);
+    int st = orc_quantize_with_scales_f32(xf, rows, cols, fmt, block, rot, scales, G, codes);
+    free(xf);
+    return st;
+}
+
 int orc_quantize_bf16(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int block,
                       int rot, int gmode, float* gscale, uint8_t* codes, uint8_t* scales)
 {
