@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "orc_quantize_search_bf16": (I, [P, I64, I64, I, I, I, I, I, I, P, P, P]),
             "orc_quantize_with_scales_f32": (I, [P, I64, I64, I, I, I, P, F, P]),
             "orc_quantize_with_scales_bf16": (I, [P, I64, I64, I, I, I, P, F, P]),
+            "orc_nearest_rank": (I64, [ctypes.c_double, I64]),
+            "orc_outlier_stats_bf16": (I, [P, I64, I64, ctypes.c_double, P, P]),
             "orc_block_mse_f32": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
             "orc_block_mse_bf16": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
         }
@@ -278,3 +280,19 @@ def unpack_nibbles(codes) -> np.ndarray:
     out[..., 0::2] = codes & 0xF
     out[..., 1::2] = codes >> 4
     return out
+
+
+def nearest_rank(p: float, n: int) -> int:
+    """k = ceil(p n) clamped to [1, n] (0 for n = 0): the rank of the p-quantile."""
+    return lib().orc_nearest_rank(p, n)
+
+
+def outlier_stats(xb, p: float = 0.999):
+    """Max |x|, the nearest-rank p-quantile of |x| and the per-column max |x| of
+    a 2-D bf16 tensor given as uint16 bit patterns."""
+    xb = np.ascontiguousarray(xb, dtype=np.uint16)
+    rows, cols = xb.shape
+    stats = np.zeros(2, np.float32)
+    col = np.zeros(cols, np.float32)
+    _check(lib().orc_outlier_stats_bf16(_ptr(xb), rows, cols, p, _ptr(stats), _ptr(col)), "outlier_stats")
+    return float(stats[0]), float(stats[1]), col

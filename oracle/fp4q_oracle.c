@@ -618,3 +618,56 @@ int orc_block_mse_bf16(const uint16_t* x, const uint8_t* codes, const uint8_t* s
     free(xf);
     return st;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Activation outlier statistics ([D] Methodology and Results C: the Max and  */
+/* the 99.9th percentile of the activations, and their ratio, per            */
+/* projection).  The pages define neither the percentile nor whether signs    */
+/* count; the reading taken here: statistics of the magnitudes |x|, and the  */
+/* p-quantile by nearest rank: with the magnitudes sorted ascending,          */
+/* a_1 <= ... <= a_N, it is a_k for k = ceil(p N) (p N in fp64, k clamped to  */
+/* [1, N]), a value that occurs in the tensor.  Per-channel maxima are the    */
+/* largest |x| of each column of the [rows][cols] = [tokens][channels]        */
+/* matrix.                                                                    */
+
+static int cmp_float_asc(const void* a, const void* b)
+{
+    float x = *(const float*)a, y = *(const float*)b;
+    return (x > y) - (x < y);
+}
+
+int64_t orc_nearest_rank(double p, int64_t n)
+{
+    if (n <= 0) return 0;
+    double t = ceil(p * (double)n);
+    int64_t k = (int64_t)t;
+    if (k < 1) k = 1;
+    if (k > n) k = n;
+    return k;
+}
+
+int orc_outlier_stats_bf16(const uint16_t* x, int64_t rows, int64_t cols, double p, float* stats,
+                           float* col_absmax)
+{
+    if (rows < 0 || cols < 0) return ORC_ESHAPE;
+    if (!(p > 0.0 && p <= 1.0) || !stats) return ORC_EARG;
+    const int64_t n = rows * cols;
+    if (col_absmax)
+        for (int64_t c = 0; c < cols; ++c) col_absmax[c] = 0.0f;
+    if (n == 0) {
+        stats[0] = 0.0f;
+        stats[1] = 0.0f;
+        return ORC_OK;
+    }
+    float* a = (float*)malloc((size_t)n * sizeof(float));
+    if (!a) return ORC_ENOMEM;
+    for (int64_t i = 0; i < n; ++i) {
+        a[i] = fabsf(orc_bf16_to_f32(x[i]));
+        if (col_absmax && a[i] > col_absmax[i % cols]) col_absmax[i % cols] = a[i];
+    }
+    qsort(a, (size_t)n, sizeof(float), cmp_float_asc);
+    stats[0] = a[n - 1];
+    stats[1] = a[orc_nearest_rank(p, n) - 1];
+    free(a);
+    return ORC_OK;
+}
