@@ -54,7 +54,18 @@ def parse_args(argv=None):
                     help="measure the MSE with its own pass over x (fp4q_quantize + fp4q_block_mse + fp4q_dequantize)")
     ap.add_argument("--separate-dequant", action="store_true",
                     help="dequantize with its own pass over the codes (fp4q_quantize_mse + fp4q_dequantize)")
-    return ap.parse_args(argv)
+    ap.add_argument("--scale-search", default=None, metavar="BELOW,ABOVE",
+                    help="MSE-optimised block scales: try BELOW codes below and ABOVE codes above the "
+                         "max-rule code (fp4q_quantize_search + fp4q_block_mse + fp4q_dequantize)")
+    ap.add_argument("--outlier-stats", type=float, default=None, metavar="P",
+                    help="add the activation outlier statistics (max, nearest-rank P-quantile of |x|, channel "
+                         "maxima: fp4q_outlier_stats) to every tensor of the step")
+    args = ap.parse_args(argv)
+    args.search = None
+    if args.scale_search:
+        below, above = (int(v) for v in args.scale_search.split(","))
+        args.search = (below, above)
+    return args
 
 
 def dist_env():
@@ -116,6 +127,8 @@ def bytes_per_element(block: int):
     return {
         "amax": 2.0,
         "quantize": 2.0 + 0.5 + 1.0 / block,
+        "quantize_search": 2.0 + 0.5 + 1.0 / block,
+        "outlier_stats": 2.0,
         "quantize_mse": 2.0 + 0.5 + 1.0 / block + 4.0 / block,
         "quantize_mse_dequantize": 2.0 + 0.5 + 1.0 / block + 4.0 / block + 2.0,
         "dequantize": 0.5 + 1.0 / block + 2.0,
@@ -133,7 +146,8 @@ class Pipeline:
     """
 
 
-    def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False):
+    def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False, search=None,
+                 outlier_p=None):
         import torch
         self.fq, self.items, self.device = fq, items, device
         L = fq.lib()
@@ -142,6 +156,7 @@ class Pipeline:
         # [amax, G] of every tensor in one buffer, cleared by one fill at the start of each step
         self.gs_all = torch.zeros((len(items), 2), dtype=torch.float32, device=device)
         self.any_comp = any(gm == COMP for *_, gm in items)
+        separate_mse = separate_mse or search is not None     # the search has no fused MSE pass
         for ti, (label, x, fmt, block, rot, gmode) in enumerate(items):
             rows, cols = x.shape
             b = dict(
@@ -155,6 +170,11 @@ class Pipeline:
                                device=device),
             )
             self.bufs.append(b)
+            if outlier_p is not None:
+                b["ostats"] = torch.empty((2,), dtype=torch.float32, device=device)
+                b["ocols"] = torch.empty((cols,), dtype=torch.float32, device=device)
+                b["ows"] = torch.empty((fq.lib().fp4q_outlier_stats_workspace_size(),), dtype=torch.uint8,
+                                       device=device)
             p = {k: v.data_ptr() for k, v in b.items()}
             comp = gmode == COMP
             # per-tensor scale: the amax pass writes gscale[0]; the quantizer derives G from it
@@ -162,10 +182,21 @@ class Pipeline:
             gq = p["gscale"] if comp else None
             g = p["gscale"] + 4 if comp else None
             seq = []
+            if outlier_p is not None:
+                seq.append(("outlier_stats", L.fp4q_outlier_stats, (x.data_ptr(), rows, cols, float(outlier_p),
+                                                                    p["ostats"], p["ocols"], p["ows"],
+                                                                    b["ows"].numel(), sh)))
             if comp:
                 seq.append(("amax", L.fp4q_tensor_amax_accumulate, (x.data_ptr(), rows, cols, rot, p["gscale"], sh)))
             gm = FROM_AMAX if comp else NONE
-            if separate_mse:
+            if search is not None:
+                seq.append(("quantize_search", L.fp4q_quantize_search,
+                            (x.data_ptr(), rows, cols, fmt, block, rot, gm, search[0], search[1], p["codes"],
+                             p["scales"], gq, sh)))
+                seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
+                                                            fmt, block, rot, p["bm"], p["terms"], p["ws"],
+                                                            b["ws"].numel(), sh)))
+            elif separate_mse:
                 seq.append(("quantize", L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot, gm,
                                                           p["codes"], p["scales"], gq, sh)))
                 seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
@@ -188,7 +219,8 @@ class Pipeline:
         # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel, + dequantized output),
         # [block MSE], [dequantize]
         self.launches_per_step = sum(1 + (1 if gm == COMP else 0) + (2 if separate_mse else 0)
-                                     + (1 if separate_dequant and not separate_mse else 0) for *_, gm in items)
+                                     + (1 if separate_dequant and not separate_mse else 0)
+                                     + (2 if outlier_p is not None else 0) for *_, gm in items)
         self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
 
     def step(self, stream, ev=None):
@@ -288,10 +320,11 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def csrc_hash() -> str:
+def csrc_hash(files=None) -> str:
+    """Hash of the named kernel sources (all of csrc/ when files is None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "microscaling_fp4_quantization_block_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files if files is not None else os.listdir(d)):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -304,7 +337,7 @@ def ncu_traffic(kernel: str, workload: str):
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             t = json.load(f)
         e = t[workload][kernel]
-        if e.get("csrc_sha") != csrc_hash():
+        if e.get("csrc_sha") != csrc_hash(e.get("csrc_files")):
             return None
         return float(e["dram_bytes_per_element"])
     except Exception:
@@ -312,14 +345,20 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 # --------------------------------------------------------------------------- CPU baseline (oracle)
-def oracle_sample_step(items_cpu):
-    """The oracle over host tensors: quantize, dequantize, block MSE."""
+def oracle_sample_step(items_cpu, search=None, outlier_p=None):
+    """The oracle over host tensors: quantize (max rule, or the scale search),
+    dequantize, block MSE."""
     import numpy as np
     import oracle
     n = 0
     for label, xb, fmt, block, rot, gmode in items_cpu:
         rows, cols = xb.shape
-        codes, scales, G = oracle.quantize(xb, fmt, block, rot, gmode)
+        if outlier_p is not None:
+            oracle.outlier_stats(xb, outlier_p)
+        if search is None:
+            codes, scales, G = oracle.quantize(xb, fmt, block, rot, gmode)
+        else:
+            codes, scales, G = oracle.quantize_search(xb, fmt, block, rot, gmode, 1.0, search[0], search[1])
         oracle.dequantize(codes, scales, G, rows, cols, fmt, block, 0)
         oracle.block_mse(xb, codes, scales, G, fmt, block, rot)
         n += xb.size
@@ -356,12 +395,12 @@ def cpu_baseline(name, args):
     """Oracle throughput on ~args.cpu_seconds of single-threaded CPU work."""
     probe = cpu_sample_items(name, args, 1_000_000)
     t0 = time.perf_counter()
-    n = oracle_sample_step(probe)
+    n = oracle_sample_step(probe, args.search, args.outlier_stats)
     rate = n / max(time.perf_counter() - t0, 1e-9)
     target = int(min(rate * args.cpu_seconds, 2_000_000_000))
     items = cpu_sample_items(name, args, target)
     t0 = time.perf_counter()
-    n = oracle_sample_step(items)
+    n = oracle_sample_step(items, args.search, args.outlier_stats)
     dt = time.perf_counter() - t0
     return {"value": n / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} elements: the first rows of each of the {len(items)} tensors, same recipe, "
@@ -377,11 +416,11 @@ def run_reference(args):
     per_step = 6_000_000 if args.workload == "nvfp4_qwen25_7b_mlp" else 2_000_000
     items = cpu_sample_items(args.workload, args, per_step)
     for _ in range(args.warmup):
-        oracle_sample_step(items)
+        oracle_sample_step(items, args.search, args.outlier_stats)
     t0 = time.perf_counter()
     n = 0
     for _ in range(args.steps):
-        n += oracle_sample_step(items)
+        n += oracle_sample_step(items, args.search, args.outlier_stats)
     dt = time.perf_counter() - t0
     value = n / dt / 1e9
     line = {"metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -389,6 +428,8 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": args.workload, "elements_per_step": int(n // args.steps),
+                       "block_scales": "max rule" if args.search is None else
+                                       f"MSE search: max-rule code, {args.search[1]} above, {args.search[0]} below",
                        "note": "the CPU oracle (single-threaded C) on a bounded sample of the workload"},
             "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
                              "sample": f"{n // args.steps} elements per step: the first rows of every tensor"},
@@ -417,7 +458,7 @@ def main(argv=None):
     stream = torch.cuda.Stream(device)
     stream.wait_stream(torch.cuda.current_stream())
     pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse,
-                    separate_dequant=args.separate_dequant)
+                    separate_dequant=args.separate_dequant, search=args.search, outlier_p=args.outlier_stats)
     in_l2 = sum(x.numel() * 2 for _, x, *_ in items) < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
 
@@ -511,6 +552,10 @@ def main(argv=None):
                    "format": {U4: "NVFP4 b16 UE4M3", E8: "MXFP4 b32 E8M0"}[items[0][2]] +
                              (" + FP32 per-tensor scale" if items[0][5] == COMP else ""),
                    "rot": items[0][4], "elements_per_step": elements_step,
+                   "block_scales": "max rule" if args.search is None else
+                                   f"MSE search: max-rule code, {args.search[1]} above, {args.search[0]} below",
+                   "outlier_stats": None if args.outlier_stats is None else
+                                    f"max, P{100 * args.outlier_stats:g} of |x| and channel maxima per tensor",
                    "l2": "L2 flushed between steps (512 MiB write)" if in_l2 else
                          f"inputs larger than L2 ({elements_step * 2 / 1e9:.2f} GB bf16 per step)",
                    "parallelism": f"{world} independent replica(s), no data-path collective",

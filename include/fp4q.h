@@ -112,6 +112,28 @@ FP4Q_API int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, i
                   int gmode, uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
 /*
+ * fp4q_quantize_search -- fp4q_quantize with MSE-optimised block scales
+ * ("Bridging the Gap", s3, MR-GPTQ item 2: scales chosen to minimise the
+ * squared reconstruction error rather than by the max rule).  The pages give
+ * no procedure; this call tries, per block, the max-rule code s0, then
+ * s0+1 .. s0+above, then s0-1 .. s0-below (codes outside the format's finite
+ * range skipped: E8M0 0..254, UE4M3 0..0x7E, UE5M3 0..0xFE) and keeps the code
+ * of least error; a later candidate wins only with a strictly smaller error,
+ * so ties keep the earlier code.  The error of a code is the fp32 sum over the
+ * block of d*d, d = fp32(y - v), v = fp32(decode(nibble) S) (0 when S = 0),
+ * each term added with one rounding; the sum's order is the kernel's, so a
+ * choice between two codes whose errors agree to fp32 rounding may differ from
+ * an element-order sum.  The nibbles are those fp4q_quantize computes for the
+ * chosen S.  below, above: 0 .. FP4Q_SEARCH_MAX (0, 0 is fp4q_quantize).
+ * Other arguments, G handling and errors as for fp4q_quantize;
+ * FP4Q_ERR_UNSUPPORTED for a window out of range.
+ */
+#define FP4Q_SEARCH_MAX 16
+FP4Q_API int fp4q_quantize_search(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                  int gmode, int below, int above, uint8_t* codes, uint8_t* scales,
+                                  float* gscale, void* stream);
+
+/*
  * fp4q_tensor_amax -- amax = max |y| over the whole (optionally rotated)
  * tensor, written as one float.  This is the first half of the per-tensor
  * scale of COMPUTE mode ("Finer is better?", Results: UE4M3 with a dynamic
@@ -214,6 +236,40 @@ FP4Q_API int fp4q_quantize_mse_dequantize(const void* x, int64_t rows, int64_t c
  * shape (host only; at most 128 KiB + 16): the completion counter and the
  * per-CTA partials. */
 FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block);
+
+/*
+ * fp4q_outlier_stats -- activation outlier statistics ("Diagnosing FP4
+ * inference", Methodology and Results C: the maximum and the 99.9th percentile
+ * of a projection's activations, and their ratio).  The pages define neither
+ * the percentile nor whether signs count; this call takes magnitudes and the
+ * nearest rank:
+ *  x          bf16 [rows][cols] = [tokens][channels] (device, 16-byte aligned);
+ *             cols a multiple of 8.  Inputs must be finite.
+ *  p          quantile in (0, 1], for instance 0.999.
+ *  stats      out (device, 2 floats): stats[0] = max |x|; stats[1] = the k-th
+ *             smallest |x|, k = ceil(p * rows*cols) evaluated in double and
+ *             clamped to [1, rows*cols] (a value present in x).  Both 0 for an
+ *             empty tensor.
+ *  col_absmax out (device, cols floats) or NULL: the largest |x| of each column.
+ *  workspace  device scratch of at least fp4q_outlier_stats_workspace_size()
+ *             bytes (8-byte aligned): two histograms over the 2^15 bf16
+ *             magnitude patterns and a control word, cleared by the call.
+ * Results are exact (integer counts over bf16 patterns).  The call zeroes its
+ * outputs and the workspace on the stream.  Below 2^22 elements it makes one
+ * histogram pass over x.  Larger tensors get three passes:
+ *  - a histogram of a sample of rows sets a threshold below the quantile;
+ *  - a pass over x counts only the magnitudes at or above the threshold and
+ *    takes the channel maxima;
+ *  - a further pass, which returns at once unless the rank turned out to lie
+ *    below the threshold, counts the rest.
+ * Each pass is followed by a single-CTA scan.  Errors: FP4Q_ERR_SHAPE
+ * (cols % 8), FP4Q_ERR_UNSUPPORTED (p outside (0, 1]), FP4Q_ERR_NULL,
+ * FP4Q_ERR_ALIGN, FP4Q_ERR_WORKSPACE.
+ */
+#define FP4Q_OUTLIER_WS_BYTES (2 * 32768 * 8 + 16)
+FP4Q_API size_t fp4q_outlier_stats_workspace_size(void);
+FP4Q_API int fp4q_outlier_stats(const void* x, int64_t rows, int64_t cols, double p, float* stats,
+                                float* col_absmax, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * fp4q_block_mse_noalloc -- fp4q_block_mse without a workspace argument, for

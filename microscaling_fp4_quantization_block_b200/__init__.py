@@ -44,6 +44,9 @@ def _load() -> ctypes.CDLL:
     P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     sig = {
         "fp4q_quantize": (I, [P, I64, I64, I, I, I, I, P, P, P, P]),
+        "fp4q_quantize_search": (I, [P, I64, I64, I, I, I, I, I, I, P, P, P, P]),
+        "fp4q_outlier_stats": (I, [P, I64, I64, ctypes.c_double, P, P, P, SZ, P]),
+        "fp4q_outlier_stats_workspace_size": (SZ, []),
         "fp4q_tensor_amax": (I, [P, I64, I64, I, P, P]),
         "fp4q_tensor_amax_accumulate": (I, [P, I64, I64, I, P, P]),
         "fp4q_global_scale": (I, [P, P, P]),
@@ -141,6 +144,58 @@ def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
                             _ptr(gscale), _stream(stream))
     _check(st, "fp4q_quantize")
     return codes, scales, gscale
+
+
+def fp4q_quantize_search(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none", below: int = 1,
+                         above: int = 1, codes: Optional[torch.Tensor] = None,
+                         scales: Optional[torch.Tensor] = None, gscale: Optional[torch.Tensor] = None,
+                         stream=None) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """fp4q_quantize with MSE-optimised block scales: per block the max-rule code,
+    then up to `above` codes above and `below` below it are tried, and the code
+    of least squared error is kept.  Returns (codes, scales, gscale)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    fmt, gmode = _fmt(fmt), _gmode(gmode)
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((rows, cols // block if block else 0), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode == FP4Q_GLOBAL_FROM_AMAX:
+        raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
+    if gscale is None and gmode != FP4Q_GLOBAL_NONE:
+        gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    _need_cuda(codes, scales, gscale)
+    st = lib().fp4q_quantize_search(_ptr(x), rows, cols, fmt, block, rot, gmode, below, above, _ptr(codes),
+                                    _ptr(scales), _ptr(gscale), _stream(stream))
+    _check(st, "fp4q_quantize_search")
+    return codes, scales, gscale
+
+
+def fp4q_outlier_stats(x: torch.Tensor, p: float = 0.999, channels: bool = True,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Activation outlier statistics of a 2-D bf16 CUDA tensor [tokens, channels]:
+    returns (stats, col_absmax) with stats = [max |x|, nearest-rank p-quantile of
+    |x|] (a 2-float CUDA tensor) and the per-channel maxima (or None)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    dev = x.device
+    stats = torch.empty((2,), dtype=torch.float32, device=dev)
+    col = torch.empty((cols,), dtype=torch.float32, device=dev) if channels else None
+    ws_bytes = lib().fp4q_outlier_stats_workspace_size()
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    _need_cuda(workspace)
+    st = lib().fp4q_outlier_stats(_ptr(x), rows, cols, float(p), _ptr(stats), _ptr(col), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "fp4q_outlier_stats")
+    return stats, col
 
 
 def fp4q_tensor_amax(x: torch.Tensor, rot: int = 0, amax: Optional[torch.Tensor] = None,

@@ -193,8 +193,11 @@ const char* fp4q_status_string(int status)
     }
 }
 
-int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
-                  uint8_t* codes, uint8_t* scales, float* gscale, void* stream)
+// fp4q_quantize and fp4q_quantize_search: the max rule, or (search) the
+// scale search over below / above neighbouring codes.
+static int quantize_impl(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                         uint8_t* codes, uint8_t* scales, float* gscale, bool search, int below, int above,
+                         void* stream)
 {
     int64_t n = 0;
     int st = check_shape(rows, cols, fmt, block, rot, &n);
@@ -230,7 +233,25 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
     p.scales = scales;
     set_global(gmode, gscale, &p.gsrc, &p.gdst);
     rotation_constants(rot, &p.c_hi, &p.c_lo);
+    if (search) {
+        p.below = below;
+        p.above = above;
+        return cuda_status(launch_quantize_search(fmt, block, rot, p, s));
+    }
     return cuda_status(launch_quantize(fmt, block, rot, false, p, nullptr, s));
+}
+
+int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                  uint8_t* codes, uint8_t* scales, float* gscale, void* stream)
+{
+    return quantize_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, false, 0, 0, stream);
+}
+
+int fp4q_quantize_search(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                         int below, int above, uint8_t* codes, uint8_t* scales, float* gscale, void* stream)
+{
+    if (below < 0 || below > FP4Q_SEARCH_MAX || above < 0 || above > FP4Q_SEARCH_MAX) return FP4Q_ERR_UNSUPPORTED;
+    return quantize_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, true, below, above, stream);
 }
 
 int fp4q_quantize_mse(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
@@ -298,6 +319,27 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gs
     p.y = y;
     rotation_constants(rot, &p.c_hi, &p.c_lo);
     return cuda_status(launch_dequantize(block, rot, out_dtype == FP4Q_OUT_F32, p, as_stream(stream)));
+}
+
+size_t fp4q_outlier_stats_workspace_size(void) { return (size_t)FP4Q_OUTLIER_WS_BYTES; }
+
+int fp4q_outlier_stats(const void* x, int64_t rows, int64_t cols, double p, float* stats, float* col_absmax,
+                       void* workspace, size_t ws_bytes, void* stream)
+{
+    if (rows < 0 || cols < 0 || cols % 8 != 0) return FP4Q_ERR_SHAPE;
+    if (cols != 0 && rows > INT64_MAX / 4 / cols) return FP4Q_ERR_SHAPE;
+    if (!(p > 0.0 && p <= 1.0)) return FP4Q_ERR_UNSUPPORTED;
+    if (!stats || !workspace) return FP4Q_ERR_NULL;
+    if (ws_bytes < (size_t)FP4Q_OUTLIER_WS_BYTES) return FP4Q_ERR_WORKSPACE;
+    if (!aligned(stats, 4) || !aligned(workspace, 8) || (col_absmax && !aligned(col_absmax, 4)))
+        return FP4Q_ERR_ALIGN;
+    const int64_t n = rows * cols;
+    if (n > 0) {
+        if (!x) return FP4Q_ERR_NULL;
+        if (!aligned(x, 16)) return FP4Q_ERR_ALIGN;
+    }
+    return cuda_status(launch_outlier_stats(static_cast<const uint16_t*>(x), rows, cols, p, stats, col_absmax,
+                                            workspace, as_stream(stream)));
 }
 
 size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int block)

@@ -83,6 +83,32 @@ __device__ __forceinline__ void stg256(void* p, uint32_t a, uint32_t b, uint32_t
                  : "memory");
 }
 
+// ---------------------------------------------------------------- L2 eviction priority
+// A cache policy under which the lines an access allocates in L2 are the
+// first to go.  Outputs, and the last read of an input, use it so that they
+// do not push out input lines that a later pass of the same step will read.
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void stg128(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "r"(a), "r"(b), "r"(c),
+                 "r"(d), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ void stg256(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                       uint32_t f, uint32_t g, uint32_t h, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8}, %9;" ::"l"(p), "r"(a), "r"(b),
+                 "r"(c), "r"(d), "r"(e), "r"(f), "r"(g), "r"(h), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void stg64(void* p, uint32_t a, uint32_t b)
 {
     asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
@@ -101,6 +127,13 @@ __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.lau
 __device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr, uint32_t src_bytes)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr), "l"(gptr), "r"(src_bytes)
+                 : "memory");
+}
+// The same copy, its L2 lines allocated under the cache policy pol.
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr, uint32_t src_bytes, uint64_t pol)
+{
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_addr), "l"(gptr),
+                 "r"(src_bytes), "l"(pol)
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }

@@ -86,8 +86,10 @@ struct Ring {
     // all) into stage s.  Bytes at or past nbytes are never read: a chunk
     // that straddles the end copies its valid prefix, and the rest, like every
     // chunk past the end, is zero-filled.
+    // With EF the copies allocate their L2 lines evict-first (policy pol).
+    template <bool EF = false>
     __device__ __forceinline__ void issue(const uint8_t* __restrict__ src, int64_t nbytes, int64_t off, int s,
-                                          int lane) const
+                                          int lane, uint64_t pol = 0) const
     {
         const uint32_t sb = base + (uint32_t)(s * TILE_BYTES);
         const uint8_t* g = src + off + 16 * lane;
@@ -95,8 +97,11 @@ struct Ring {
 #pragma unroll
             for (int h = 0; h < UPS; ++h)
 #pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    cp_async16(sb + (uint32_t)(h * SUB_BYTES) + wr[c], g + h * SUB_BYTES + 512 * c, 16u);
+                for (int c = 0; c < CPL; ++c) {
+                    const uint32_t d = sb + (uint32_t)(h * SUB_BYTES) + wr[c];
+                    if constexpr (EF) cp_async16(d, g + h * SUB_BYTES + 512 * c, 16u, pol);
+                    else cp_async16(d, g + h * SUB_BYTES + 512 * c, 16u);
+                }
         } else {
 #pragma unroll
             for (int h = 0; h < UPS; ++h)
@@ -135,10 +140,11 @@ __device__ __forceinline__ R warp_ring(uint8_t* smem)
 
 // Ring pipeline driver: calls body(tile, stage) for every tile of this warp,
 // with the tile's input resident in the ring.  NSTAGE - 1 tiles are in flight.
-template <typename R, typename Body>
+// EF: the copies allocate their L2 lines evict-first (policy pol).
+template <bool EF = false, typename R, typename Body>
 __device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __restrict__ src, int64_t nbytes,
                                              int64_t n_tiles, int64_t warp, int64_t n_warps, int lane,
-                                             Body&& body)
+                                             Body&& body, uint64_t pol = 0)
 {
     constexpr int NS = R::NSTAGE;
     const int64_t step = n_warps * R::TILE_BYTES;
@@ -146,7 +152,7 @@ __device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __res
     int64_t off_issue = warp * R::TILE_BYTES;
 #pragma unroll
     for (int s = 0; s < NS - 1; ++s) {
-        if (t_issue < n_tiles) ring.issue(src, nbytes, off_issue, s, lane);
+        if (t_issue < n_tiles) ring.template issue<EF>(src, nbytes, off_issue, s, lane, pol);
         cp_async_commit();
         t_issue += n_warps;
         off_issue += step;
@@ -154,7 +160,7 @@ __device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __res
     int stage = 0;
     for (int64_t t = warp; t < n_tiles; t += n_warps) {
         const int s_new = stage == 0 ? NS - 1 : stage - 1;          // the slot read last iteration
-        if (t_issue < n_tiles) ring.issue(src, nbytes, off_issue, s_new, lane);
+        if (t_issue < n_tiles) ring.template issue<EF>(src, nbytes, off_issue, s_new, lane, pol);
         cp_async_commit();
         t_issue += n_warps;
         off_issue += step;
@@ -452,12 +458,58 @@ struct QuantParams {
     double* terms;         // fused MSE: the four tensor terms
     float* gdst;           // G from the tensor maximum: *gsrc is that maximum, G is written here
     uint16_t* y;           // fused MSE with dequantized output: n bf16 values
+    int below, above;      // scale search: codes tried below / above the max-rule code
 };
+
+// Store a unit's code word (16 bytes; with EF evict-first in L2, for codes
+// that nothing reads again in the step) and its blocks' scale bytes; a unit
+// that reaches past n stores only its valid prefix.
+template <int B, int K, bool EF>
+__device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, const uint32_t (&cw)[EPT / 8],
+                                           const uint32_t (&code)[UnitShape<B, K>::NB], int lane, uint64_t pol)
+{
+    using S = UnitShape<B, K>;
+    constexpr int NB = S::NB;
+    const int64_t e0 = u * EPT;
+    if (e0 >= p.n) return;
+    uint8_t* cdst = p.codes + e0 / 2;
+    if (e0 + EPT <= p.n) {
+        if constexpr (EF) stg128(cdst, cw[0], cw[1], cw[2], cw[3], pol);
+        else stg128(cdst, cw[0], cw[1], cw[2], cw[3]);
+    } else {
+        const int nbytes = (int)((p.n - e0) / 2);
+#pragma unroll
+        for (int k = 0; k < EPT / 8; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (4 * k + j < nbytes) cdst[4 * k + j] = (uint8_t)(cw[k] >> (8 * j));
+    }
+    if constexpr (S::LPB > 1) {
+        if ((lane % S::LPB) == 0) p.scales[e0 / B] = (uint8_t)code[0];
+    } else {
+        const int64_t b0 = e0 / B;
+        const int64_t nblk = p.n / B;
+        if (e0 + EPT <= p.n) {
+            if constexpr (NB == 1) {
+                p.scales[b0] = (uint8_t)code[0];
+            } else if constexpr (NB == 2) {
+                *reinterpret_cast<uint16_t*>(p.scales + b0) = (uint16_t)(code[0] | (code[1] << 8));
+            } else {
+                *reinterpret_cast<uint32_t*>(p.scales + b0) =
+                    code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24);
+            }
+        } else {
+#pragma unroll
+            for (int bi = 0; bi < NB; ++bi)
+                if (b0 + bi < nblk) p.scales[b0 + bi] = (uint8_t)code[bi];
+        }
+    }
+}
 
 template <int FMT, int B, int K, bool MSE, bool DQ>
 __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
                                               int lane, const ScaleConsts& kc, const float2* tab, float nz,
-                                              double (&acc)[3])
+                                              double (&acc)[3], uint64_t pol)
 {
     using S = UnitShape<B, K>;
     constexpr int NB = S::NB, BE = S::BE;
@@ -541,7 +593,8 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
 #pragma unroll
                         for (int j = 0; j < 4; ++j) ypend[j] = yw[j];
                     } else {
-                        stg256(p.y + ew - 8, ypend[0], ypend[1], ypend[2], ypend[3], yw[0], yw[1], yw[2], yw[3]);
+                        stg256(p.y + ew - 8, ypend[0], ypend[1], ypend[2], ypend[3], yw[0], yw[1], yw[2], yw[3],
+                               pol);
                     }
                 } else {
 #pragma unroll
@@ -597,39 +650,7 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
     }
 
     // ---- stores
-    const int64_t e0 = u * EPT;
-    if (e0 >= p.n) return;
-    uint8_t* cdst = p.codes + e0 / 2;
-    if (e0 + EPT <= p.n) {
-        stg128(cdst, cw[0], cw[1], cw[2], cw[3]);
-    } else {
-        const int nbytes = (int)((p.n - e0) / 2);
-#pragma unroll
-        for (int k = 0; k < EPT / 8; ++k)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (4 * k + j < nbytes) cdst[4 * k + j] = (uint8_t)(cw[k] >> (8 * j));
-    }
-    if constexpr (S::LPB > 1) {
-        if ((lane % S::LPB) == 0) p.scales[e0 / B] = (uint8_t)code[0];
-    } else {
-        const int64_t b0 = e0 / B;
-        const int64_t nblk = p.n / B;
-        if (e0 + EPT <= p.n) {
-            if constexpr (NB == 1) {
-                p.scales[b0] = (uint8_t)code[0];
-            } else if constexpr (NB == 2) {
-                *reinterpret_cast<uint16_t*>(p.scales + b0) = (uint16_t)(code[0] | (code[1] << 8));
-            } else {
-                *reinterpret_cast<uint32_t*>(p.scales + b0) =
-                    code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24);
-            }
-        } else {
-#pragma unroll
-            for (int bi = 0; bi < NB; ++bi)
-                if (b0 + bi < nblk) p.scales[b0 + bi] = (uint8_t)code[bi];
-        }
-    }
+    store_unit<B, K, DQ>(p, u, cw, code, lane, pol);
 }
 
 // Two CTAs per SM (up to 128 registers) unless the kernel fits three without
@@ -666,16 +687,174 @@ __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quant
     const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
     double acc[3] = {0.0, 0.0, 0.0};        // squared errors: all, block maxima, zero-rounded blocks
 
-    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
-                 [&](int64_t t, int s) {
-                     uint32_t w[EPT / 2];
-                     ring.read(s, 0, w);
-                     quantize_unit<FMT, B, K, MSE, DQ>(p, t * 32 + lane, w, lane, kc, tab, nz, acc);
-                 });
+    // Evict-first in L2 for what the step does not read again, so that it does
+    // not push out lines that are: x where this is its last read (MSE fused), and
+    // the codes and dequantized values of the fused dequantizing kernel.
+    const uint64_t pol = l2_evict_first();
+    stream_tiles<MSE>(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
+                            [&](int64_t t, int s) {
+                                uint32_t w[EPT / 2];
+                                ring.read(s, 0, w);
+                                quantize_unit<FMT, B, K, MSE, DQ>(p, t * 32 + lane, w, lane, kc, tab, nz, acc, pol);
+                            },
+                            pol);
     if constexpr (MSE) {
         cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
         finish_partials(p.partials, p.done, p.n, p.terms);
     }
+}
+
+// ---------------------------------------------------------------- MSE-optimised block scales
+// "Bridging the Gap", s3 (MR-GPTQ, MSE-optimised grids): each block's scale is
+// the code of least squared reconstruction error among the max-rule code s0,
+// s0+1 .. s0+above and s0-1 .. s0-below, tried in that order; codes outside the
+// finite range are skipped and a candidate wins only with a strictly smaller
+// error, so ties keep the earlier code.  The error of a candidate is the fp32
+// sum of d^2, d = fp32(y - v), v = fp32(decode(code) S) (0 for S = 0).
+
+// Block scale and its reciprocal for a candidate code, and whether the code is
+// a finite scale of the format.  UE formats read the per-tensor table; E8M0
+// scales are powers of two with exact reciprocals (2^-127 for byte 254).
+template <int FMT>
+__device__ __forceinline__ bool candidate_scale(int c, const float2* tab, float& S, float& R)
+{
+    if constexpr (FMT == kE8M0) {
+        if (c < 0 || c > 254) return false;
+        S = e8m0_decode((uint32_t)c);
+        R = c == 254 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(254 - c) << 23);
+        return true;
+    } else {
+        if (c < 0 || c > (FMT == kUE4M3 ? 0x7e : 0xfe)) return false;
+        const float2 e = tab[c];
+        S = e.x;
+        R = e.y;
+        return true;
+    }
+}
+
+template <int FMT, int B, int K>
+__device__ __forceinline__ void search_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2], int lane,
+                                            const ScaleConsts& kc, const float2* tab, float nz, uint64_t pol)
+{
+    using S = UnitShape<B, K>;
+    constexpr int NB = S::NB, BE = S::BE;
+    f32x2 v[EPT / 2];
+    unpack_unit(w, v);
+    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+    float m[NB];
+    if constexpr (K == 0) block_max_words<B>(w, m);
+    else block_max<B, K>(v, m);
+
+    float s0S[NB], s0R[NB];
+    uint32_t s0[NB];
+    unit_scales<FMT, NB>(m, kc, tab, s0, s0S, s0R);
+
+    uint32_t best[NB];
+    float best_err[NB];
+    uint32_t cw[EPT / 8];
+    const f32x2 nz2 = pk(nz, nz);
+    const int ncand = 1 + p.above + p.below;
+    for (int j = 0; j < ncand; ++j) {
+        const int delta = j == 0 ? 0 : (j <= p.above ? j : p.above - j);
+        float Sc[NB], Rc[NB];
+        bool ok[NB], quot_ok[NB];
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) {
+            ok[bi] = candidate_scale<FMT>((int)s0[bi] + delta, tab, Sc[bi], Rc[bi]);
+            if (!ok[bi]) Sc[bi] = Rc[bi] = 0.0f;
+            // the remainder-corrected quotient needs S in its range and |m / S| <= 2^60
+            quot_ok[bi] = FMT == kE8M0 || (__fmul_rn(m[bi], Rc[bi]) <= kQuotMax);
+        }
+        uint32_t cj[EPT / 8];
+        f32x2 bsum[NB];
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) bsum[bi] = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int k = 0; k < EPT / 8; ++k) {
+            const int bi = (8 * k) / BE;
+            const f32x2* vk = v + 4 * k;
+            uint32_t h[4];
+            if (Sc[bi] == 0.0f) {
+                cj[k] = 0u;                                         // zero-rounded: every v is 0
+#pragma unroll
+                for (int q = 0; q < 4; ++q) h[q] = 0u;
+            } else if (FMT == kE8M0) {
+                const f32x2 r = pk(Rc[bi], Rc[bi]);
+                cj[k] = pack_pairs_dec(mul2(vk[0], r), mul2(vk[1], r), mul2(vk[2], r), mul2(vk[3], r), h);
+            } else if (quot_ok[bi]) {
+                const f32x2 R2 = pk(Rc[bi], Rc[bi]), nS2 = pk(-Sc[bi], -Sc[bi]);
+                cj[k] = pack_pairs_dec(div2_cr(vk[0], R2, nS2), div2_cr(vk[1], R2, nS2), div2_cr(vk[2], R2, nS2),
+                                       div2_cr(vk[3], R2, nS2), h);
+            } else {
+                cj[k] = pack_pairs_div(vk[0], vk[1], vk[2], vk[3], Sc[bi]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t hh;
+                    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+                        : "=r"(hh) : "r"((cj[k] >> (8 * q)) & 0xffu));
+                    h[q] = hh;
+                }
+            }
+            const f32x2 s2 = pk(Sc[bi], Sc[bi]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __half2 hh = *reinterpret_cast<__half2*>(&h[q]);
+                const f32x2 g = pk(__low2float(hh), __high2float(hh));
+                const f32x2 d = sub2(vk[q], fma2(g, s2, nz2));        // y - fp32(g S)
+                bsum[bi] = fma2(d, d, bsum[bi]);
+            }
+        }
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi) {
+            float se, so;
+            upk(bsum[bi], se, so);
+            float e = __fadd_rn(se, so);
+            if constexpr (S::LPB > 1) e = group_sum<S::LPB>(e);
+            const bool take = j == 0 || (ok[bi] && e < best_err[bi]);
+            if (take) {
+                best_err[bi] = e;
+                best[bi] = (uint32_t)((int)s0[bi] + delta);
+#pragma unroll
+                for (int k = 0; k < EPT / 8; ++k)
+                    if ((8 * k) / BE == bi) cw[k] = cj[k];
+            }
+        }
+    }
+    store_unit<B, K, false>(p, u, cw, best, lane, pol);
+}
+
+template <int FMT, int B, int K>
+__global__ void __launch_bounds__(kThreads, 2) search_kernel(QuantParams p)
+{
+    pdl_wait();
+    pdl_release();
+    extern __shared__ __align__(128) uint8_t smem_ring[];
+    const int lane = threadIdx.x & 31;
+    const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const XRing ring = warp_ring<XRing>(smem_ring);
+
+    float G = 1.0f;
+    if (FMT != kE8M0 && p.gsrc != nullptr) {
+        G = *p.gsrc;
+        if (p.gdst != nullptr) {
+            G = G > 0.0f ? __fdiv_rn(G, 2688.0f) : 1.0f;
+            if (blockIdx.x == 0 && threadIdx.x == 0) *p.gdst = G;
+        }
+    }
+    const ScaleConsts kc = scale_consts(G);
+    __shared__ float2 tab[256];
+    if constexpr (FMT != kE8M0) fill_scale_table<FMT>(tab, G);
+    __syncthreads();
+    const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
+    // x and the codes are read again by the MSE and dequantize passes: default L2 policy
+    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
+                 [&](int64_t t, int s) {
+                     uint32_t w[EPT / 2];
+                     ring.read(s, 0, w);
+                     search_unit<FMT, B, K>(p, t * 32 + lane, w, lane, kc, tab, nz, 0);
+                 });
 }
 
 // ---------------------------------------------------------------- per-tensor amax
@@ -797,6 +976,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
 {
     pdl_wait();
     pdl_release();
+    const uint64_t pol = l2_evict_first();        // outputs: not read again in the step
     constexpr int NSB = DeqScales<B>::NSB;
     constexpr int EPB = B <= DPL ? B : DPL;                       // elements of a block in a lane
     using R = Ring<64, 1>;                                        // 64 code bytes per lane per tile
@@ -853,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
                         upk(v[4 * k + 3], a[6], a[7]);
                         stg256(dst + 8 * k, __float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
                                __float_as_uint(a[3]), __float_as_uint(a[4]), __float_as_uint(a[5]),
-                               __float_as_uint(a[6]), __float_as_uint(a[7]));
+                               __float_as_uint(a[6]), __float_as_uint(a[7]), pol);
                     }
                 } else {
 #pragma unroll
@@ -879,7 +1059,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DequantParams p)
                         o[j] = *reinterpret_cast<uint32_t*>(&hb);
                     }
                     if (full) {
-                        stg256(dst + 8 * k, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                        stg256(dst + 8 * k, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7], pol);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
@@ -962,6 +1142,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_il_kernel(DequantParams p
     static_assert(K == 0 || K == kDqChunk, "interleaved chunks hold rotation runs of at most 16");
     pdl_wait();
     pdl_release();
+    const uint64_t pol = l2_evict_first();        // outputs: not read again in the step
     using D = DqStage<B>;
     extern __shared__ __align__(128) uint8_t smem_ring[];
     __shared__ float tab[256];                                   // block scale by code
@@ -1026,10 +1207,10 @@ __global__ void __launch_bounds__(kThreads) dequantize_il_kernel(DequantParams p
                 for (int j = 0; j < 8; ++j) upk(v[j], a[2 * j], a[2 * j + 1]);
                 if (full) {
                     stg256(dst, __float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]), __float_as_uint(a[3]),
-                           __float_as_uint(a[4]), __float_as_uint(a[5]), __float_as_uint(a[6]), __float_as_uint(a[7]));
+                           __float_as_uint(a[4]), __float_as_uint(a[5]), __float_as_uint(a[6]), __float_as_uint(a[7]), pol);
                     stg256(dst + 8, __float_as_uint(a[8]), __float_as_uint(a[9]), __float_as_uint(a[10]),
                            __float_as_uint(a[11]), __float_as_uint(a[12]), __float_as_uint(a[13]), __float_as_uint(a[14]),
-                           __float_as_uint(a[15]));
+                           __float_as_uint(a[15]), pol);
                 } else {
                     for (int j = 0; j < kDqChunk; ++j)
                         if (e0 + j < p.n) dst[j] = a[j];
@@ -1045,7 +1226,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_il_kernel(DequantParams p
                 }
                 uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.y) + e0);
                 if (full) {
-                    stg256(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                    stg256(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7], pol);
                 } else {
                     for (int j = 0; j < 8; ++j)
                         if (e0 + 2 * j < p.n) dst[j] = o[j];

@@ -31,7 +31,13 @@ cudaError_t launch_quantize_ue4m3(int B, int K, bool mse, const QuantParams& p, 
 cudaError_t launch_quantize_ue5m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 // pdl: launch with programmatic dependent launch (never right after the memset
 // that zeroes the maximum's slot, which must complete first).
+// Quantize with MSE-optimised block scales (p.below / p.above candidate codes).
+cudaError_t launch_quantize_search(int fmt, int B, int K, const QuantParams& p, cudaStream_t s);
 cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl);
+// Outlier statistics: zeroes the histogram (workspace), stats and col_absmax,
+// then one histogram pass over x and a one-CTA scan.
+cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, double p, float* stats,
+                                 float* col_absmax, void* workspace, cudaStream_t s);
 cudaError_t launch_dequantize(int B, int K, bool f32out, const DequantParams& p, cudaStream_t s);
 cudaError_t launch_block_mse(int B, int K, const MseParams& p, int* grid_out, cudaStream_t s);
 

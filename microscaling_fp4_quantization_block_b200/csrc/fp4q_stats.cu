@@ -1,0 +1,333 @@
+// fp4q_stats.cu -- activation outlier statistics ("Diagnosing FP4 inference",
+// Methodology and Results C: the maximum and the 99.9th percentile of the
+// activations, whose ratio separates the down projection from the others).
+//
+// max |x|, the nearest-rank p-quantile of |x| (the k-th smallest magnitude,
+// k = ceil(p n)) and the per-channel maxima of a bf16 [rows][cols] tensor.
+// A bf16 magnitude has 2^15 bit patterns, and non-negative bf16 values order
+// like their patterns, so a histogram over the patterns gives the quantile
+// exactly.
+//
+// Only the magnitudes near the quantile need counting one by one.  A tensor of
+// at least kDirectElems elements is therefore done in three steps:
+//  1. a histogram of every s-th row estimates the quantile, and sets a
+//     threshold L a safe margin below it;
+//  2. the main pass histograms only magnitudes >= L (a few in a thousand for
+//     P99.9) and takes every channel maximum; the magnitudes below L are then
+//     n minus the histogram's total;
+//  3. if rank k falls among the counted magnitudes the answer is exact;
+//     otherwise (L was not below the quantile) a pass gated on a device flag
+//     adds the magnitudes below L, and the scan is repeated on the full
+//     histogram.
+// Smaller tensors take one full histogram pass.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp4q_device.cuh"
+#include "fp4q_launch.h"
+
+namespace fp4q {
+namespace {
+
+constexpr int kBins = 1 << 15;               // bf16 magnitude patterns
+constexpr int kStatThreads = 1024;
+constexpr int kHistSmem = kBins * 4;          // 128 KiB of per-CTA counts
+constexpr int64_t kDirectElems = int64_t(1) << 22;
+constexpr int64_t kSampleElems = int64_t(1) << 20;   // at least this many in the estimate
+constexpr int kMaxSampleStride = 16;
+
+struct StatsCtl {
+    uint32_t L;          // magnitudes >= L are counted by the main pass
+    uint32_t fallback;   // set when the rank lies below L
+};
+
+enum : int { kAllBins = 0, kFromL = 1, kBelowLIfNeeded = 2 };
+
+struct StatsParams {
+    const uint16_t* x;
+    int64_t rows;              // rows visited: 0, row_step, 2 row_step, ... (rows of them)
+    int64_t row_step;
+    int64_t g;                 // 16-byte chunks per row (cols / 8)
+    int64_t r;                 // visited rows between a thread's consecutive rows
+    int64_t T;                 // working threads: g * r
+    unsigned long long* hist;  // [kBins] counts
+    unsigned int* colmax;      // [cols] fp32 bits of the channel maxima (zeroed) or nullptr
+    const StatsCtl* ctl;
+    int mode;
+};
+
+__device__ __forceinline__ uint4 ldg128_stream(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Count the 8 magnitudes of a chunk that lie in [lo, lo + span) and fold them
+// into this thread's 8 channel maxima.
+__device__ __forceinline__ void count_chunk(const uint4& v, uint32_t* sh, uint32_t lo, uint32_t span,
+                                            uint32_t (&cm)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t a = w[k] & 0x7fffu, b = (w[k] >> 16) & 0x7fffu;
+        if (a - lo < span) atomicAdd(sh + a, 1u);
+        if (b - lo < span) atomicAdd(sh + b, 1u);
+        cm[2 * k] = max(cm[2 * k], a);
+        cm[2 * k + 1] = max(cm[2 * k + 1], b);
+    }
+}
+
+// Thread t owns the 8 channels of chunk t % g in visited rows t / g, t / g + r,
+// ...: consecutive threads read consecutive 16-byte chunks of a row, and a
+// thread's channel maxima stay in registers until the end.
+__global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsParams p)
+{
+    pdl_wait();
+    pdl_release();
+    uint32_t lo = 0u, hi = (uint32_t)kBins;
+    if (p.mode == kFromL) {
+        lo = p.ctl->L;
+    } else if (p.mode == kBelowLIfNeeded) {
+        if (!p.ctl->fallback) return;
+        hi = p.ctl->L;
+    }
+    extern __shared__ __align__(16) uint32_t sh_hist[];
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) sh_hist[i] = 0u;
+    __syncthreads();
+    const uint32_t span = hi - lo;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t cm[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (tid < p.T) {
+        const int64_t c8 = tid % p.g;
+        const uint4* base = reinterpret_cast<const uint4*>(p.x) + c8;
+        const int64_t stride = p.row_step * p.g;                  // chunks between visited rows
+        int64_t j = tid / p.g;
+        for (; j + 3 * p.r < p.rows; j += 4 * p.r) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = ldg128_stream(base + (j + u * p.r) * stride);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) count_chunk(v[u], sh_hist, lo, span, cm);
+        }
+        for (; j < p.rows; j += p.r) count_chunk(ldg128_stream(base + j * stride), sh_hist, lo, span, cm);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
+        const uint32_t c = sh_hist[i];
+        if (c) atomicAdd(p.hist + i, (unsigned long long)c);
+    }
+    if (tid < p.T && p.colmax) {
+        unsigned int* dst = p.colmax + 8 * (tid % p.g);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (cm[j]) atomicMax(dst + j, cm[j] << 16);     // |x| as fp32 bits: orders as integers
+    }
+}
+
+// Block-wide scan helpers for the single-CTA kernels: thread t owns bins
+// [32 t, 32 t + 32); after the call scan[t] holds the inclusive prefix count.
+constexpr int kPer = kBins / kStatThreads;
+
+__device__ __forceinline__ unsigned long long prefix_counts(const unsigned long long* hist,
+                                                            unsigned long long* scan, int* top)
+{
+    const int t = threadIdx.x;
+    unsigned long long sum = 0;
+    int hi = -1;
+#pragma unroll 8
+    for (int j = 0; j < kPer; ++j) {                             // independent loads, issued together
+        const unsigned long long c = hist[kPer * t + j];
+        sum += c;
+        if (c) hi = kPer * t + j;
+    }
+    if (t == 0) *top = -1;
+    scan[t] = sum;
+    __syncthreads();
+    if (hi >= 0) atomicMax(top, hi);
+    for (int d = 1; d < kStatThreads; d <<= 1) {                 // Hillis-Steele
+        const unsigned long long add = t >= d ? scan[t - d] : 0ull;
+        __syncthreads();
+        scan[t] += add;
+        __syncthreads();
+    }
+    return sum;
+}
+
+// The bin holding the rank-th smallest counted magnitude (1 <= rank <= total),
+// found by the thread whose bins contain it; returns -1 in the other threads.
+__device__ __forceinline__ int bin_of_rank(const unsigned long long* hist, const unsigned long long* scan,
+                                           unsigned long long own, unsigned long long rank)
+{
+    const int t = threadIdx.x;
+    const unsigned long long incl = scan[t], excl = incl - own;
+    if (!(excl < rank && rank <= incl)) return -1;
+    unsigned long long c[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) c[j] = hist[kPer * t + j];
+    unsigned long long run = excl;
+    int bin = -1;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        run += c[j];
+        if (bin < 0 && run >= rank) bin = kPer * t + j;
+    }
+    return bin;
+}
+
+struct ThresholdParams {
+    const unsigned long long* shist;   // histogram of the sampled rows
+    double p;
+    StatsCtl* ctl;
+};
+
+// L = the sampled magnitude at fraction p_low = 1 - 2(1 - p) - 8 sd of the
+// sample, sd = sqrt(p (1 - p) / n_s) (0 when p_low * n_s < 1).
+__global__ void __launch_bounds__(kStatThreads) outlier_threshold_kernel(ThresholdParams q)
+{
+    pdl_wait();
+    pdl_release();
+    __shared__ unsigned long long scan[kStatThreads];
+    __shared__ int top;
+    const unsigned long long own = prefix_counts(q.shist, scan, &top);
+    const unsigned long long ns = scan[kStatThreads - 1];
+    double plow = 1.0 - 2.0 * (1.0 - q.p) - 8.0 * sqrt(q.p * (1.0 - q.p) / (double)(ns > 0 ? ns : 1));
+    if (plow < 0.0) plow = 0.0;
+    const unsigned long long rank = (unsigned long long)floor(plow * (double)ns);
+    if (threadIdx.x == 0) {
+        q.ctl->fallback = 0u;
+        if (rank < 1) q.ctl->L = 0u;
+    }
+    if (rank >= 1) {
+        const int b = bin_of_rank(q.shist, scan, own, rank);
+        if (b >= 0) q.ctl->L = (uint32_t)b;
+    }
+}
+
+struct FinalizeParams {
+    const unsigned long long* hist;
+    int64_t n;
+    double p;
+    float* stats;
+    StatsCtl* ctl;     // nullptr: hist is complete (direct path)
+    int phase;         // 0: hist holds the magnitudes >= L; 1: hist is complete (gated on the fallback flag)
+};
+
+// stats[0] = the largest magnitude present, stats[1] = the magnitude of rank
+// k = ceil(p n) (clamped to [1, n]).
+__global__ void __launch_bounds__(kStatThreads) outlier_finalize_kernel(FinalizeParams q)
+{
+    pdl_wait();
+    pdl_release();
+    if (q.phase == 1 && q.ctl && !q.ctl->fallback) return;
+    __shared__ unsigned long long scan[kStatThreads];
+    __shared__ int top;
+    const unsigned long long own = prefix_counts(q.hist, scan, &top);
+    const unsigned long long counted = scan[kStatThreads - 1];
+    long long k = (long long)ceil(q.p * (double)q.n);
+    if (k < 1) k = 1;
+    if (k > q.n) k = q.n;
+    const unsigned long long below = (unsigned long long)q.n - counted;   // magnitudes not counted (< L)
+    if (q.phase == 0 && (unsigned long long)k <= below) {
+        if (threadIdx.x == 0) q.ctl->fallback = 1u;      // the rank lies below L: count those too
+        return;
+    }
+    const int b = bin_of_rank(q.hist, scan, own, (unsigned long long)k - below);
+    if (b >= 0) q.stats[1] = __uint_as_float((uint32_t)b << 16);
+    if (threadIdx.x == 0) q.stats[0] = top >= 0 ? __uint_as_float((uint32_t)top << 16) : 0.0f;
+}
+
+int hist_grid(StatsParams& prm, int sms)
+{
+    const int64_t target = (int64_t)(sms > 0 ? sms : 1) * kStatThreads;
+    int64_t r = target / prm.g;
+    if (r < 1) r = 1;
+    if (r > prm.rows) r = prm.rows;
+    prm.r = r;
+    prm.T = prm.g * r;
+    const int64_t blocks = (prm.T + kStatThreads - 1) / kStatThreads;
+    return blocks > 0x7fffffff ? -1 : (int)blocks;
+}
+
+}  // namespace
+
+cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, double p, float* stats,
+                                 float* col_absmax, void* workspace, cudaStream_t s)
+{
+    auto* hist = static_cast<unsigned long long*>(workspace);
+    auto* shist = hist + kBins;
+    auto* ctl = reinterpret_cast<StatsCtl*>(shist + kBins);
+    cudaError_t e = cudaMemsetAsync(hist, 0, 2 * sizeof(unsigned long long) * kBins + sizeof(StatsCtl), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, 2 * sizeof(float), s);
+    if (e == cudaSuccess && col_absmax) e = cudaMemsetAsync(col_absmax, 0, sizeof(float) * (size_t)cols, s);
+    if (e != cudaSuccess) return e;
+    const int64_t n = rows * cols;
+    if (n == 0) return cudaSuccess;
+
+    static bool opted[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !opted[dev]) {
+        e = cudaFuncSetAttribute(outlier_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kHistSmem);
+        if (e != cudaSuccess) return e;
+        opted[dev] = true;
+    }
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+    StatsParams main{};
+    main.x = x;
+    main.rows = rows;
+    main.row_step = 1;
+    main.g = cols / 8;
+    main.hist = hist;
+    main.colmax = reinterpret_cast<unsigned int*>(col_absmax);
+    main.ctl = ctl;
+    const int main_blocks = hist_grid(main, sms);
+    if (main_blocks < 0) return cudaErrorInvalidValue;
+
+    if (n < kDirectElems) {                                   // one full histogram pass
+        main.mode = kAllBins;
+        outlier_hist_kernel<<<main_blocks, kStatThreads, kHistSmem, s>>>(main);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, nullptr, 1});
+    }
+
+    // 1. sample every s-th row (at least kSampleElems elements) and set L
+    int64_t stride = n / kSampleElems;
+    if (stride > kMaxSampleStride) stride = kMaxSampleStride;
+    if (stride > rows) stride = rows;
+    if (stride < 1) stride = 1;
+    StatsParams smp = main;
+    smp.rows = (rows + stride - 1) / stride;
+    smp.row_step = stride;
+    smp.hist = shist;
+    smp.colmax = nullptr;
+    smp.mode = kAllBins;
+    const int smp_blocks = hist_grid(smp, sms);
+    outlier_hist_kernel<<<smp_blocks, kStatThreads, kHistSmem, s>>>(smp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(outlier_threshold_kernel, 1, kStatThreads, 0, s, ThresholdParams{shist, p, ctl})) !=
+        cudaSuccess)
+        return e;
+    // 2. magnitudes >= L, every channel maximum
+    main.mode = kFromL;
+    if ((e = launch_pdl(outlier_hist_kernel, main_blocks, kStatThreads, kHistSmem, s, main)) != cudaSuccess)
+        return e;
+    if ((e = launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, ctl, 0})) !=
+        cudaSuccess)
+        return e;
+    // 3. only if the rank lay below L: the rest of the histogram, and the scan again
+    StatsParams rest = main;
+    rest.colmax = nullptr;
+    rest.mode = kBelowLIfNeeded;
+    if ((e = launch_pdl(outlier_hist_kernel, main_blocks, kStatThreads, kHistSmem, s, rest)) != cudaSuccess)
+        return e;
+    return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, ctl, 1});
+}
+
+}  // namespace fp4q

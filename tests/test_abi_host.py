@@ -110,6 +110,33 @@ def test_dequantize_and_mse_reject_bad_arguments(fp4q):
     assert L.fp4q_global_scale(A32 + 2, A32, None) == -3
 
 
+def test_search_and_outlier_stats_reject_bad_arguments(fp4q):
+    L = fp4q.lib()
+    qs = L.fp4q_quantize_search
+    assert qs(A32, 4, 64, 1, 16, 0, 0, -1, 1, A32, A32, None, None) == -4         # window below 0
+    assert qs(A32, 4, 64, 1, 16, 0, 0, 1, 17, A32, A32, None, None) == -4         # window above 16
+    assert qs(A32, 4, 48, 0, 32, 0, 0, 1, 1, A32, A32, None, None) == -2          # 48 % 32
+    assert qs(A32, 4, 64, 0, 32, 0, 1, 1, 1, A32, A32, A32, None) == -4           # MX has no tensor scale
+    assert qs(None, 4, 64, 1, 16, 0, 0, 1, 1, A32, A32, None, None) == -1
+    assert qs(A32 + 16, 4, 64, 1, 16, 0, 0, 1, 1, A32, A32, None, None) == -3
+    assert qs(None, 0, 64, 1, 16, 0, 0, 3, 2, None, None, None, None) == 0        # empty: nothing enqueued
+    ws = L.fp4q_outlier_stats_workspace_size()
+    assert ws == 2 * 32768 * 8 + 16
+    os_ = L.fp4q_outlier_stats
+    assert os_(A32, 4, 60, 0.999, A32, None, A32, ws, None) == -2                 # cols % 8
+    assert os_(A32, -1, 64, 0.999, A32, None, A32, ws, None) == -2
+    for p in (0.0, -0.1, 1.01, float("nan")):
+        assert os_(A32, 4, 64, p, A32, None, A32, ws, None) == -4
+    assert os_(A32, 4, 64, 0.999, None, None, A32, ws, None) == -1                # stats
+    assert os_(A32, 4, 64, 0.999, A32, None, None, ws, None) == -1                # workspace
+    assert os_(None, 4, 64, 0.999, A32, None, A32, ws, None) == -1                # x
+    assert os_(A32, 4, 64, 0.999, A32, None, A32, ws - 8, None) == -6
+    assert os_(A32 + 8, 4, 64, 0.999, A32, None, A32, ws, None) == -3             # x 16-aligned
+    assert os_(A32, 4, 64, 0.999, A32 + 2, None, A32, ws, None) == -3
+    assert os_(A32, 4, 64, 0.999, A32, A32 + 2, A32, ws, None) == -3
+    assert os_(A32, 4, 64, 0.999, A32, None, A32 + 4, ws, None) == -3
+
+
 def test_workspace_size_is_bounded(fp4q):
     L = fp4q.lib()
     small = L.fp4q_block_mse_workspace_size(1, 16, 16)
