@@ -218,9 +218,13 @@ class Pipeline:
         self.elements = sum(x.numel() for _, x, *_ in items)
         # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel, + dequantized output),
         # [block MSE], [dequantize]
+        # outlier statistics: one histogram pass and a scan below 2^22 elements; above, a sampled
+        # pass, the threshold scan, the main pass, a scan, and a pass and a scan that return at once
+        # unless the threshold missed
         self.launches_per_step = sum(1 + (1 if gm == COMP else 0) + (2 if separate_mse else 0)
                                      + (1 if separate_dequant and not separate_mse else 0)
-                                     + (2 if outlier_p is not None else 0) for *_, gm in items)
+                                     + (0 if outlier_p is None else (6 if x.numel() >= (1 << 22) else 2))
+                                     for _, x, *_, gm in items)
         self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
 
     def step(self, stream, ev=None):

@@ -66,19 +66,30 @@ __device__ __forceinline__ uint4 ldg128_stream(const void* p)
     return r;
 }
 
-// Count the 8 magnitudes of a chunk that lie in [lo, lo + span) and fold them
-// into this thread's 8 channel maxima.
-__device__ __forceinline__ void count_chunk(const uint4& v, uint32_t* sh, uint32_t lo, uint32_t span,
-                                            uint32_t (&cm)[8])
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
 {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Fold a chunk's 8 magnitudes into this thread's channel maxima (two channels
+// per word, packed), and count those in [lo, lo + span).  A chunk whose largest
+// magnitude is below lo -- almost every chunk when only the top of the
+// distribution is counted -- costs a few packed maxima and one branch.
+__device__ __forceinline__ void count_chunk(const uint4& v, uint32_t* sh, uint32_t lo, uint32_t span,
+                                            uint32_t (&cmw)[4])
+{
+    const uint32_t w[4] = {v.x & 0x7fff7fffu, v.y & 0x7fff7fffu, v.z & 0x7fff7fffu, v.w & 0x7fff7fffu};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cmw[k] = max_u16x2(cmw[k], w[k]);
+    const uint32_t m = max_u16x2(max_u16x2(w[0], w[1]), max_u16x2(w[2], w[3]));
+    if (max(m & 0xffffu, m >> 16) < lo) return;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const uint32_t a = w[k] & 0x7fffu, b = (w[k] >> 16) & 0x7fffu;
+        const uint32_t a = w[k] & 0xffffu, b = w[k] >> 16;
         if (a - lo < span) atomicAdd(sh + a, 1u);
         if (b - lo < span) atomicAdd(sh + b, 1u);
-        cm[2 * k] = max(cm[2 * k], a);
-        cm[2 * k + 1] = max(cm[2 * k + 1], b);
     }
 }
 
@@ -101,7 +112,7 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
     __syncthreads();
     const uint32_t span = hi - lo;
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    uint32_t cm[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    uint32_t cmw[4] = {0u, 0u, 0u, 0u};                           // channel maxima, two per word
     if (tid < p.T) {
         const int64_t c8 = tid % p.g;
         const uint4* base = reinterpret_cast<const uint4*>(p.x) + c8;
@@ -112,9 +123,9 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
 #pragma unroll
             for (int u = 0; u < 4; ++u) v[u] = ldg128_stream(base + (j + u * p.r) * stride);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) count_chunk(v[u], sh_hist, lo, span, cm);
+            for (int u = 0; u < 4; ++u) count_chunk(v[u], sh_hist, lo, span, cmw);
         }
-        for (; j < p.rows; j += p.r) count_chunk(ldg128_stream(base + j * stride), sh_hist, lo, span, cm);
+        for (; j < p.rows; j += p.r) count_chunk(ldg128_stream(base + j * stride), sh_hist, lo, span, cmw);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
@@ -124,8 +135,10 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
     if (tid < p.T && p.colmax) {
         unsigned int* dst = p.colmax + 8 * (tid % p.g);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (cm[j]) atomicMax(dst + j, cm[j] << 16);     // |x| as fp32 bits: orders as integers
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = (j & 1) ? cmw[j >> 1] >> 16 : cmw[j >> 1] & 0xffffu;
+            if (c) atomicMax(dst + j, c << 16);              // |x| as fp32 bits: orders as integers
+        }
     }
 }
 

@@ -147,3 +147,34 @@ def test_search_empty_and_errors(fq):
         fq.fp4q_quantize_search(x, U4, 16, 0, "none", 17, 0)
     with pytest.raises(fq.Fp4qError):
         fq.fp4q_quantize_search(x, U4, 16, 0, "none", 0, -1)
+
+
+def test_search_full_size_sampled_rows(fq):
+    """The scale search on a whole Qwen2.5-7B MLP weight (gate 18944 x 3584,
+    sigma 0.005, the benchmark's first tensor) in the benchmark's configuration: NVFP4 b16 with the per-tensor
+    scale derived from the tensor maximum, window 2 below / 1 above.  Sampled
+    rows against the oracle with the same G (blocks never cross a row)."""
+    name, x = next(iter(workloads.nvfp4_mlp_tensors(device="cuda")))
+    amax = fq.fp4q_tensor_amax(x)
+    gs = torch.zeros((2,), dtype=torch.float32, device="cuda")
+    gs[0] = amax[0]
+    c1, s1, _ = fq.fp4q_quantize_search(x, U4, 16, 0, "from_amax", 2, 1, gscale=gs)
+    c0, s0, _ = fq.fp4q_quantize(x, U4, 16, 0, "from_amax", gscale=gs.clone())
+    torch.cuda.synchronize()
+    G = float(gs[1].item())
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, x.shape[0] - 1], rng.integers(0, x.shape[0], 40)]))
+    ri = torch.from_numpy(rows).cuda()
+    xb = bf16_bits(x[ri])
+    g_codes, g_scales = c1[ri].cpu().numpy(), s1[ri].cpu().numpy()
+    oc, os_, _ = oracle.quantize_search(xb, U4, 16, 0, GIVEN, G, 2, 1)
+    d = g_scales.astype(np.int64) - s0[ri].cpu().numpy().astype(np.int64)
+    assert ((d >= -2) & (d <= 1)).all()
+    e_gpu, oc_g = _errors(xb, g_scales, G, U4, 16, 0)
+    e_orc, _ = _errors(xb, os_, G, U4, 16, 0)
+    differ = g_scales != os_
+    tol = 2.0 * (16 + 4) * 2.0 ** -24
+    assert not (differ & (np.abs(e_gpu - e_orc) > tol * np.maximum(e_gpu, e_orc) + 1e-300)).any()
+    assert differ.sum() <= max(2, 1e-3 * differ.size)
+    assert np.array_equal(g_codes, oc_g)
+    assert (g_scales != s0[ri].cpu().numpy()).mean() > 0.01     # the search moves a share of the blocks
