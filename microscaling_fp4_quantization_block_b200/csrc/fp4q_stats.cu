@@ -118,12 +118,12 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
         const uint4* base = reinterpret_cast<const uint4*>(p.x) + c8;
         const int64_t stride = p.row_step * p.g;                  // chunks between visited rows
         int64_t j = tid / p.g;
-        for (; j + 3 * p.r < p.rows; j += 4 * p.r) {
-            uint4 v[4];
+        for (; j + 7 * p.r < p.rows; j += 8 * p.r) {                // 8 loads in flight
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = ldg128_stream(base + (j + u * p.r) * stride);
+            for (int u = 0; u < 8; ++u) v[u] = ldg128_stream(base + (j + u * p.r) * stride);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) count_chunk(v[u], sh_hist, lo, span, cmw);
+            for (int u = 0; u < 8; ++u) count_chunk(v[u], sh_hist, lo, span, cmw);
         }
         for (; j < p.rows; j += p.r) count_chunk(ldg128_stream(base + j * stride), sh_hist, lo, span, cmw);
     }
@@ -142,54 +142,91 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
     }
 }
 
-// Block-wide scan helpers for the single-CTA kernels: thread t owns bins
-// [32 t, 32 t + 32); after the call scan[t] holds the inclusive prefix count.
-constexpr int kPer = kBins / kStatThreads;
+// Histogram scans for the single-CTA kernels.  Warp w owns bins [1024 w,
+// 1024 w + 1024) and reads them with coalesced loads; the 32 warp totals are
+// scanned once, and only the warp whose range holds a rank looks inside it.
+struct ScanSmem {
+    unsigned long long wtot[32];    // per-warp totals
+    unsigned long long wexcl[32];   // counts before each warp's range
+    unsigned long long total;
+    int top;                        // largest nonzero bin, -1 if none
+    int found;
+};
 
-__device__ __forceinline__ unsigned long long prefix_counts(const unsigned long long* hist,
-                                                            unsigned long long* scan, int* top)
+__device__ __forceinline__ unsigned long long warp_sum(unsigned long long v)
 {
-    const int t = threadIdx.x;
-    unsigned long long sum = 0;
-    int hi = -1;
-#pragma unroll 8
-    for (int j = 0; j < kPer; ++j) {                             // independent loads, issued together
-        const unsigned long long c = hist[kPer * t + j];
-        sum += c;
-        if (c) hi = kPer * t + j;
-    }
-    if (t == 0) *top = -1;
-    scan[t] = sum;
-    __syncthreads();
-    if (hi >= 0) atomicMax(top, hi);
-    for (int d = 1; d < kStatThreads; d <<= 1) {                 // Hillis-Steele
-        const unsigned long long add = t >= d ? scan[t - d] : 0ull;
-        __syncthreads();
-        scan[t] += add;
-        __syncthreads();
-    }
-    return sum;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    return v;
 }
 
-// The bin holding the rank-th smallest counted magnitude (1 <= rank <= total),
-// found by the thread whose bins contain it; returns -1 in the other threads.
-__device__ __forceinline__ int bin_of_rank(const unsigned long long* hist, const unsigned long long* scan,
-                                           unsigned long long own, unsigned long long rank)
+__device__ __forceinline__ unsigned long long warp_inclusive_scan(unsigned long long v, int lane)
 {
-    const int t = threadIdx.x;
-    const unsigned long long incl = scan[t], excl = incl - own;
-    if (!(excl < rank && rank <= incl)) return -1;
-    unsigned long long c[kPer];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) c[j] = hist[kPer * t + j];
-    unsigned long long run = excl;
-    int bin = -1;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        run += c[j];
-        if (bin < 0 && run >= rank) bin = kPer * t + j;
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long t = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += t;
     }
-    return bin;
+    return v;
+}
+
+// Totals of the histogram: fills sm and returns the total count (every thread).
+__device__ __forceinline__ unsigned long long hist_summary(const unsigned long long* hist, ScanSmem& sm)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const unsigned long long* hw = hist + 1024 * w;
+    unsigned long long s = 0;
+    int hi = -1;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {                               // coalesced, independent loads
+        const unsigned long long c = hw[32 * i + l];
+        s += c;
+        if (c) hi = 1024 * w + 32 * i + l;
+    }
+    s = warp_sum(s);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, d));
+    if (threadIdx.x == 0) sm.top = -1;
+    __syncthreads();
+    if (l == 0) {
+        sm.wtot[w] = s;
+        atomicMax(&sm.top, hi);
+    }
+    __syncthreads();
+    if (w == 0) {
+        const unsigned long long t = sm.wtot[l];
+        const unsigned long long inc = warp_inclusive_scan(t, l);
+        sm.wexcl[l] = inc - t;
+        if (l == 31) sm.total = inc;
+    }
+    __syncthreads();
+    return sm.total;
+}
+
+// The bin holding the rank-th smallest counted magnitude, 1 <= rank <= total
+// (every thread gets it; hist_summary must have filled sm).
+__device__ __forceinline__ int bin_at_rank(const unsigned long long* hist, unsigned long long rank, ScanSmem& sm)
+{
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (threadIdx.x == 0) sm.found = -1;
+    __syncthreads();
+    const unsigned long long ex = sm.wexcl[w];
+    if (rank > ex && rank <= ex + sm.wtot[w]) {                  // one warp, uniformly
+        const unsigned long long need = rank - ex;
+        const unsigned long long* hc = hist + 1024 * w + 32 * l;  // lane l: chunk l of 32 bins
+        unsigned long long ct = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) ct += hc[j];
+        const unsigned long long inc = warp_inclusive_scan(ct, l);
+        const int c = __ffs(__ballot_sync(0xffffffffu, inc >= need)) - 1;
+        const unsigned long long before = __shfl_sync(0xffffffffu, inc - ct, c);
+        const unsigned long long v = hist[1024 * w + 32 * c + l];
+        const unsigned long long inc2 = warp_inclusive_scan(v, l);
+        const int b = __ffs(__ballot_sync(0xffffffffu, before + inc2 >= need)) - 1;
+        if (l == 0) sm.found = 1024 * w + 32 * c + b;
+    }
+    __syncthreads();
+    return sm.found;
 }
 
 struct ThresholdParams {
@@ -204,20 +241,15 @@ __global__ void __launch_bounds__(kStatThreads) outlier_threshold_kernel(Thresho
 {
     pdl_wait();
     pdl_release();
-    __shared__ unsigned long long scan[kStatThreads];
-    __shared__ int top;
-    const unsigned long long own = prefix_counts(q.shist, scan, &top);
-    const unsigned long long ns = scan[kStatThreads - 1];
+    __shared__ ScanSmem sm;
+    const unsigned long long ns = hist_summary(q.shist, sm);
     double plow = 1.0 - 2.0 * (1.0 - q.p) - 8.0 * sqrt(q.p * (1.0 - q.p) / (double)(ns > 0 ? ns : 1));
     if (plow < 0.0) plow = 0.0;
     const unsigned long long rank = (unsigned long long)floor(plow * (double)ns);
+    const int L = rank >= 1 ? bin_at_rank(q.shist, rank, sm) : 0;
     if (threadIdx.x == 0) {
+        q.ctl->L = (uint32_t)(L > 0 ? L : 0);
         q.ctl->fallback = 0u;
-        if (rank < 1) q.ctl->L = 0u;
-    }
-    if (rank >= 1) {
-        const int b = bin_of_rank(q.shist, scan, own, rank);
-        if (b >= 0) q.ctl->L = (uint32_t)b;
     }
 }
 
@@ -237,10 +269,8 @@ __global__ void __launch_bounds__(kStatThreads) outlier_finalize_kernel(Finalize
     pdl_wait();
     pdl_release();
     if (q.phase == 1 && q.ctl && !q.ctl->fallback) return;
-    __shared__ unsigned long long scan[kStatThreads];
-    __shared__ int top;
-    const unsigned long long own = prefix_counts(q.hist, scan, &top);
-    const unsigned long long counted = scan[kStatThreads - 1];
+    __shared__ ScanSmem sm;
+    const unsigned long long counted = hist_summary(q.hist, sm);
     long long k = (long long)ceil(q.p * (double)q.n);
     if (k < 1) k = 1;
     if (k > q.n) k = q.n;
@@ -249,9 +279,11 @@ __global__ void __launch_bounds__(kStatThreads) outlier_finalize_kernel(Finalize
         if (threadIdx.x == 0) q.ctl->fallback = 1u;      // the rank lies below L: count those too
         return;
     }
-    const int b = bin_of_rank(q.hist, scan, own, (unsigned long long)k - below);
-    if (b >= 0) q.stats[1] = __uint_as_float((uint32_t)b << 16);
-    if (threadIdx.x == 0) q.stats[0] = top >= 0 ? __uint_as_float((uint32_t)top << 16) : 0.0f;
+    const int b = bin_at_rank(q.hist, (unsigned long long)k - below, sm);
+    if (threadIdx.x == 0) {
+        if (b >= 0) q.stats[1] = __uint_as_float((uint32_t)b << 16);
+        q.stats[0] = sm.top >= 0 ? __uint_as_float((uint32_t)sm.top << 16) : 0.0f;
+    }
 }
 
 int hist_grid(StatsParams& prm, int sms)
