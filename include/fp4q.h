@@ -253,7 +253,8 @@ FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int bl
  *  col_absmax out (device, cols floats) or NULL: the largest |x| of each column.
  *  workspace  device scratch of at least fp4q_outlier_stats_workspace_size()
  *             bytes (8-byte aligned): two histograms over the 2^15 bf16
- *             magnitude patterns and a control word, cleared by the call.
+ *             magnitude patterns, their totals per exponent (256 each) and a
+ *             control word, cleared by the call.
  * Results are exact (integer counts over bf16 patterns).  The call zeroes its
  * outputs and the workspace on the stream.  Below 2^22 elements it makes one
  * histogram pass over x.  Larger tensors get three passes:
@@ -266,7 +267,7 @@ FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int bl
  * (cols % 8), FP4Q_ERR_UNSUPPORTED (p outside (0, 1]), FP4Q_ERR_NULL,
  * FP4Q_ERR_ALIGN, FP4Q_ERR_WORKSPACE.
  */
-#define FP4Q_OUTLIER_WS_BYTES (2 * 32768 * 8 + 16)
+#define FP4Q_OUTLIER_WS_BYTES (2 * 32768 * 8 + 2 * 256 * 8 + 16)
 FP4Q_API size_t fp4q_outlier_stats_workspace_size(void);
 FP4Q_API int fp4q_outlier_stats(const void* x, int64_t rows, int64_t cols, double p, float* stats,
                                 float* col_absmax, void* workspace, size_t ws_bytes, void* stream);

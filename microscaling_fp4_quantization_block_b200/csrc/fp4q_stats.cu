@@ -31,6 +31,7 @@ namespace fp4q {
 namespace {
 
 constexpr int kBins = 1 << 15;               // bf16 magnitude patterns
+constexpr int kBuckets = 256;                 // one per exponent field: 128 mantissa bins each
 constexpr int kStatThreads = 1024;
 constexpr int kHistSmem = kBins * 4;          // 128 KiB of per-CTA counts
 constexpr int64_t kDirectElems = int64_t(1) << 22;
@@ -52,6 +53,7 @@ struct StatsParams {
     int64_t r;                 // visited rows between a thread's consecutive rows
     int64_t T;                 // working threads: g * r
     unsigned long long* hist;  // [kBins] counts
+    unsigned long long* buck;  // [kBuckets] totals of hist's 128-bin buckets
     unsigned int* colmax;      // [cols] fp32 bits of the channel maxima (zeroed) or nullptr
     const StatsCtl* ctl;
     int mode;
@@ -132,6 +134,18 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
         const uint32_t c = sh_hist[i];
         if (c) atomicAdd(p.hist + i, (unsigned long long)c);
     }
+    {
+        // bucket totals: four threads per bucket, 32 bins each, the bin order
+        // rotated by lane so that a warp's shared reads hit 32 different banks
+        const int t = threadIdx.x, l = t & 31;
+        const uint32_t* b = sh_hist + 32 * t;                   // bins 32 t .. 32 t + 31 = part t % 4 of bucket t / 4
+        unsigned long long sum = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) sum += b[(j + l) & 31];
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if ((t & 3) == 0 && sum) atomicAdd(p.buck + (t >> 2), sum);
+    }
     if (tid < p.T && p.colmax) {
         unsigned int* dst = p.colmax + 8 * (tid % p.g);
 #pragma unroll
@@ -142,23 +156,21 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
     }
 }
 
-// Histogram scans for the single-CTA kernels.  Warp w owns bins [1024 w,
-// 1024 w + 1024) and reads them with coalesced loads; the 32 warp totals are
-// scanned once, and only the warp whose range holds a rank looks inside it.
+// Histogram scans for the single-CTA kernels.  They read the 256 bucket
+// totals (2 KiB), then the 128 bins of the one bucket that holds a rank or the
+// maximum.
 struct ScanSmem {
-    unsigned long long wtot[32];    // per-warp totals
-    unsigned long long wexcl[32];   // counts before each warp's range
+    unsigned long long bval[kBuckets];    // bucket totals
+    unsigned long long bexcl[kBuckets];   // counts before each bucket
+    unsigned long long wtot[8];           // per-warp sums of the bucket totals
+    unsigned long long wexcl[8];
     unsigned long long total;
-    int top;                        // largest nonzero bin, -1 if none
+    unsigned long long need;
+    int topb;                             // largest nonzero bucket, -1 if none
+    int top;                              // largest nonzero bin, -1 if none
+    int fb;
     int found;
 };
-
-__device__ __forceinline__ unsigned long long warp_sum(unsigned long long v)
-{
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-    return v;
-}
 
 __device__ __forceinline__ unsigned long long warp_inclusive_scan(unsigned long long v, int lane)
 {
@@ -170,34 +182,46 @@ __device__ __forceinline__ unsigned long long warp_inclusive_scan(unsigned long 
     return v;
 }
 
-// Totals of the histogram: fills sm and returns the total count (every thread).
-__device__ __forceinline__ unsigned long long hist_summary(const unsigned long long* hist, ScanSmem& sm)
+__device__ __forceinline__ int warp_max(int v)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    const unsigned long long* hw = hist + 1024 * w;
-    unsigned long long s = 0;
-    int hi = -1;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {                               // coalesced, independent loads
-        const unsigned long long c = hw[32 * i + l];
-        s += c;
-        if (c) hi = 1024 * w + 32 * i + l;
-    }
-    s = warp_sum(s);
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, d));
-    if (threadIdx.x == 0) sm.top = -1;
+    for (int d = 16; d > 0; d >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, d));
+    return v;
+}
+
+// Bucket prefix counts and the largest bin present; returns the total count.
+__device__ __forceinline__ unsigned long long hist_summary(const unsigned long long* hist,
+                                                           const unsigned long long* buck, ScanSmem& sm)
+{
+    const int t = threadIdx.x, w = t >> 5, l = t & 31;
+    if (t == 0) sm.topb = -1;
+    const unsigned long long v = t < kBuckets ? buck[t] : 0ull;
+    const unsigned long long inc = warp_inclusive_scan(v, l);
+    const int hb = warp_max(t < kBuckets && v ? t : -1);
     __syncthreads();
-    if (l == 0) {
-        sm.wtot[w] = s;
-        atomicMax(&sm.top, hi);
-    }
+    if (w < kBuckets / 32 && l == 31) sm.wtot[w] = inc;
+    if (l == 0 && hb >= 0) atomicMax(&sm.topb, hb);
     __syncthreads();
     if (w == 0) {
-        const unsigned long long t = sm.wtot[l];
-        const unsigned long long inc = warp_inclusive_scan(t, l);
-        sm.wexcl[l] = inc - t;
-        if (l == 31) sm.total = inc;
+        const unsigned long long x = l < kBuckets / 32 ? sm.wtot[l] : 0ull;
+        const unsigned long long iw = warp_inclusive_scan(x, l);
+        if (l < kBuckets / 32) sm.wexcl[l] = iw - x;
+        if (l == kBuckets / 32 - 1) sm.total = iw;
+    }
+    __syncthreads();
+    if (t < kBuckets) {
+        sm.bval[t] = v;
+        sm.bexcl[t] = sm.wexcl[w] + inc - v;
+    }
+    if (w == 0) {                                                // largest bin of the top bucket
+        int hi = -1;
+        if (sm.topb >= 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (hist[128 * sm.topb + 32 * q + l]) hi = 128 * sm.topb + 32 * q + l;
+        }
+        hi = warp_max(hi);
+        if (l == 0) sm.top = hi;
     }
     __syncthreads();
     return sm.total;
@@ -207,23 +231,39 @@ __device__ __forceinline__ unsigned long long hist_summary(const unsigned long l
 // (every thread gets it; hist_summary must have filled sm).
 __device__ __forceinline__ int bin_at_rank(const unsigned long long* hist, unsigned long long rank, ScanSmem& sm)
 {
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (threadIdx.x == 0) sm.found = -1;
+    const int t = threadIdx.x, l = t & 31;
+    if (t == 0) {                                                // in-range defaults: a rank outside
+        sm.found = -1;                                           // [1, total] cannot index past the
+        sm.fb = 0;                                               // histogram
+        sm.need = 1;
+    }
     __syncthreads();
-    const unsigned long long ex = sm.wexcl[w];
-    if (rank > ex && rank <= ex + sm.wtot[w]) {                  // one warp, uniformly
-        const unsigned long long need = rank - ex;
-        const unsigned long long* hc = hist + 1024 * w + 32 * l;  // lane l: chunk l of 32 bins
-        unsigned long long ct = 0;
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) ct += hc[j];
-        const unsigned long long inc = warp_inclusive_scan(ct, l);
-        const int c = __ffs(__ballot_sync(0xffffffffu, inc >= need)) - 1;
-        const unsigned long long before = __shfl_sync(0xffffffffu, inc - ct, c);
-        const unsigned long long v = hist[1024 * w + 32 * c + l];
-        const unsigned long long inc2 = warp_inclusive_scan(v, l);
-        const int b = __ffs(__ballot_sync(0xffffffffu, before + inc2 >= need)) - 1;
-        if (l == 0) sm.found = 1024 * w + 32 * c + b;
+    if (t < kBuckets) {
+        const unsigned long long ex = sm.bexcl[t];
+        if (rank > ex && rank <= ex + sm.bval[t]) {             // exactly one bucket
+            sm.fb = t;
+            sm.need = rank - ex;
+        }
+    }
+    __syncthreads();
+    if (t < 32) {
+        // lane l: bins 4 l .. 4 l + 3 of the bucket, in order
+        const unsigned long long* hb = hist + 128 * sm.fb + 4 * l;
+        unsigned long long c[4], s = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            c[q] = hb[q];
+            s += c[q];
+        }
+        const unsigned long long need = sm.need;
+        const unsigned long long inc = warp_inclusive_scan(s, l);
+        const int lane = __ffs(__ballot_sync(0xffffffffu, inc >= need)) - 1;
+        if (l == lane) {
+            unsigned long long run = inc - s;
+            int q = 0;
+            while (q < 3 && run + c[q] < need) run += c[q++];
+            sm.found = 128 * sm.fb + 4 * l + q;
+        }
     }
     __syncthreads();
     return sm.found;
@@ -231,6 +271,7 @@ __device__ __forceinline__ int bin_at_rank(const unsigned long long* hist, unsig
 
 struct ThresholdParams {
     const unsigned long long* shist;   // histogram of the sampled rows
+    const unsigned long long* sbuck;   // its bucket totals
     double p;
     StatsCtl* ctl;
 };
@@ -242,7 +283,7 @@ __global__ void __launch_bounds__(kStatThreads) outlier_threshold_kernel(Thresho
     pdl_wait();
     pdl_release();
     __shared__ ScanSmem sm;
-    const unsigned long long ns = hist_summary(q.shist, sm);
+    const unsigned long long ns = hist_summary(q.shist, q.sbuck, sm);
     double plow = 1.0 - 2.0 * (1.0 - q.p) - 8.0 * sqrt(q.p * (1.0 - q.p) / (double)(ns > 0 ? ns : 1));
     if (plow < 0.0) plow = 0.0;
     const unsigned long long rank = (unsigned long long)floor(plow * (double)ns);
@@ -255,6 +296,7 @@ __global__ void __launch_bounds__(kStatThreads) outlier_threshold_kernel(Thresho
 
 struct FinalizeParams {
     const unsigned long long* hist;
+    const unsigned long long* buck;
     int64_t n;
     double p;
     float* stats;
@@ -270,7 +312,7 @@ __global__ void __launch_bounds__(kStatThreads) outlier_finalize_kernel(Finalize
     pdl_release();
     if (q.phase == 1 && q.ctl && !q.ctl->fallback) return;
     __shared__ ScanSmem sm;
-    const unsigned long long counted = hist_summary(q.hist, sm);
+    const unsigned long long counted = hist_summary(q.hist, q.buck, sm);
     long long k = (long long)ceil(q.p * (double)q.n);
     if (k < 1) k = 1;
     if (k > q.n) k = q.n;
@@ -305,8 +347,10 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
 {
     auto* hist = static_cast<unsigned long long*>(workspace);
     auto* shist = hist + kBins;
-    auto* ctl = reinterpret_cast<StatsCtl*>(shist + kBins);
-    cudaError_t e = cudaMemsetAsync(hist, 0, 2 * sizeof(unsigned long long) * kBins + sizeof(StatsCtl), s);
+    auto* hbuck = shist + kBins;
+    auto* sbuck = hbuck + kBuckets;
+    auto* ctl = reinterpret_cast<StatsCtl*>(sbuck + kBuckets);
+    cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(unsigned long long) * (2 * kBins + 2 * kBuckets) + sizeof(StatsCtl), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, 2 * sizeof(float), s);
     if (e == cudaSuccess && col_absmax) e = cudaMemsetAsync(col_absmax, 0, sizeof(float) * (size_t)cols, s);
     if (e != cudaSuccess) return e;
@@ -330,6 +374,7 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
     main.row_step = 1;
     main.g = cols / 8;
     main.hist = hist;
+    main.buck = hbuck;
     main.colmax = reinterpret_cast<unsigned int*>(col_absmax);
     main.ctl = ctl;
     const int main_blocks = hist_grid(main, sms);
@@ -339,7 +384,7 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
         main.mode = kAllBins;
         outlier_hist_kernel<<<main_blocks, kStatThreads, kHistSmem, s>>>(main);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, nullptr, 1});
+        return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, hbuck, n, p, stats, nullptr, 1});
     }
 
     // 1. sample every s-th row (at least kSampleElems elements) and set L
@@ -351,19 +396,20 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
     smp.rows = (rows + stride - 1) / stride;
     smp.row_step = stride;
     smp.hist = shist;
+    smp.buck = sbuck;
     smp.colmax = nullptr;
     smp.mode = kAllBins;
     const int smp_blocks = hist_grid(smp, sms);
     outlier_hist_kernel<<<smp_blocks, kStatThreads, kHistSmem, s>>>(smp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_pdl(outlier_threshold_kernel, 1, kStatThreads, 0, s, ThresholdParams{shist, p, ctl})) !=
+    if ((e = launch_pdl(outlier_threshold_kernel, 1, kStatThreads, 0, s, ThresholdParams{shist, sbuck, p, ctl})) !=
         cudaSuccess)
         return e;
     // 2. magnitudes >= L, every channel maximum
     main.mode = kFromL;
     if ((e = launch_pdl(outlier_hist_kernel, main_blocks, kStatThreads, kHistSmem, s, main)) != cudaSuccess)
         return e;
-    if ((e = launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, ctl, 0})) !=
+    if ((e = launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, hbuck, n, p, stats, ctl, 0})) !=
         cudaSuccess)
         return e;
     // 3. only if the rank lay below L: the rest of the histogram, and the scan again
@@ -372,7 +418,7 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
     rest.mode = kBelowLIfNeeded;
     if ((e = launch_pdl(outlier_hist_kernel, main_blocks, kStatThreads, kHistSmem, s, rest)) != cudaSuccess)
         return e;
-    return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, n, p, stats, ctl, 1});
+    return launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, hbuck, n, p, stats, ctl, 1});
 }
 
 }  // namespace fp4q

@@ -121,7 +121,7 @@ def test_search_and_outlier_stats_reject_bad_arguments(fp4q):
     assert qs(A32 + 16, 4, 64, 1, 16, 0, 0, 1, 1, A32, A32, None, None) == -3
     assert qs(None, 0, 64, 1, 16, 0, 0, 3, 2, None, None, None, None) == 0        # empty: nothing enqueued
     ws = L.fp4q_outlier_stats_workspace_size()
-    assert ws == 2 * 32768 * 8 + 16
+    assert ws == 2 * 32768 * 8 + 2 * 256 * 8 + 16
     os_ = L.fp4q_outlier_stats
     assert os_(A32, 4, 60, 0.999, A32, None, A32, ws, None) == -2                 # cols % 8
     assert os_(A32, -1, 64, 0.999, A32, None, A32, ws, None) == -2
