@@ -434,6 +434,8 @@ def run_reference(args):
             "config": {"workload": args.workload, "elements_per_step": int(n // args.steps),
                        "block_scales": "max rule" if args.search is None else
                                        f"MSE search: max-rule code, {args.search[1]} above, {args.search[0]} below",
+                       "outlier_stats": None if args.outlier_stats is None else
+                                        f"max, P{100 * args.outlier_stats:g} of |x| and channel maxima per tensor",
                        "note": "the CPU oracle (single-threaded C) on a bounded sample of the workload"},
             "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
                              "sample": f"{n // args.steps} elements per step: the first rows of every tensor"},
