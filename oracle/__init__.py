@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "orc_quantize_with_scales_f32": (I, [P, I64, I64, I, I, I, P, F, P]),
             "orc_quantize_with_scales_bf16": (I, [P, I64, I64, I, I, I, P, F, P]),
             "orc_nearest_rank": (I64, [ctypes.c_double, I64]),
+            "orc_fp4_gemm": (I, [P, P, F, I64, P, P, F, I64, I64, I, I, P]),
             "orc_outlier_stats_bf16": (I, [P, I64, I64, ctypes.c_double, P, P]),
             "orc_block_mse_f32": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
             "orc_block_mse_bf16": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
@@ -296,3 +297,20 @@ def outlier_stats(xb, p: float = 0.999):
     col = np.zeros(cols, np.float32)
     _check(lib().orc_outlier_stats_bf16(_ptr(xb), rows, cols, p, _ptr(stats), _ptr(col)), "outlier_stats")
     return float(stats[0]), float(stats[1]), col
+
+
+def fp4_gemm(codes_a, scales_a, ga: float, codes_b, scales_b, gb: float, k: int, fmt: int, block: int):
+    """Y = G_A G_B sum_k q_A s_A q_B s_B (fp64, [rows_A][rows_B]) of two quantized
+    operands, each [rows][k] with blocks of `block` along k."""
+    if k <= 0:
+        raise ValueError("k must be positive")
+    codes_a = np.ascontiguousarray(codes_a, dtype=np.uint8)
+    codes_b = np.ascontiguousarray(codes_b, dtype=np.uint8)
+    scales_a = np.ascontiguousarray(scales_a, dtype=np.uint8)
+    scales_b = np.ascontiguousarray(scales_b, dtype=np.uint8)
+    m = codes_a.size * 2 // k
+    n = codes_b.size * 2 // k
+    y = np.empty((m, n), np.float64)
+    _check(lib().orc_fp4_gemm(_ptr(codes_a), _ptr(scales_a), ga, m, _ptr(codes_b), _ptr(scales_b), gb, n, k, fmt,
+                              block, _ptr(y)), "fp4_gemm")
+    return y

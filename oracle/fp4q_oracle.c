@@ -671,3 +671,40 @@ int orc_outlier_stats_bf16(const uint16_t* x, int64_t rows, int64_t cols, double
     free(a);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP4 GEMM consumer ([B] s3-4: the QuTLASS kernels take the FP4 codes and   */
+/* block scales of both operands; [D] Methodology: weights are quantized on  */
+/* the fly and dequantized for the compute).  The pages give no formula; the */
+/* reading taken here is the exact product of the two quantized operands:    */
+/*   Y[m][n] = G_A G_B sum_k q_A[m][k] s_A[m][k/b] q_B[n][k] s_B[n][k/b],     */
+/* with q the E2M1 value of a nibble and s the decoded scale byte (without   */
+/* the per-tensor scale), both operands [rows][K] row-major with blocks of b */
+/* along K, evaluated in fp64 in k order.                                    */
+
+int orc_fp4_gemm(const uint8_t* codes_a, const uint8_t* scales_a, float ga, int64_t m_rows,
+                 const uint8_t* codes_b, const uint8_t* scales_b, float gb, int64_t n_rows,
+                 int64_t k_len, int fmt, int block, double* y)
+{
+    int st = check_layout(m_rows, k_len, fmt, block, 0);
+    if (st) return st;
+    st = check_layout(n_rows, k_len, fmt, block, 0);
+    if (st) return st;
+    const int64_t nb = k_len / block;
+    const double g = (double)ga * (double)gb;
+    for (int64_t i = 0; i < m_rows; ++i) {
+        for (int64_t j = 0; j < n_rows; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < k_len; ++k) {
+                const int64_t ea = i * k_len + k, eb = j * k_len + k;
+                const uint8_t na = (uint8_t)((codes_a[ea >> 1] >> ((ea & 1) ? 4 : 0)) & 0xfu);
+                const uint8_t nbb = (uint8_t)((codes_b[eb >> 1] >> ((eb & 1) ? 4 : 0)) & 0xfu);
+                const double sa = (double)scale_of_code(fmt, scales_a[i * nb + k / block], 1.0f);
+                const double sb = (double)scale_of_code(fmt, scales_b[j * nb + k / block], 1.0f);
+                acc += (double)orc_e2m1_decode(na) * sa * (double)orc_e2m1_decode(nbb) * sb;
+            }
+            y[i * n_rows + j] = acc * g;
+        }
+    }
+    return ORC_OK;
+}
