@@ -395,8 +395,48 @@ def cpu_sample_items(name: str, args, elements_target: int):
     return out
 
 
+MAX_ORACLE_PROCS = 32
+
+
+def _oracle_init():
+    import oracle
+    oracle.lib()
+
+
+def _oracle_worker(payload):
+    items, search, outlier_p = payload
+    return oracle_sample_step(items, search, outlier_p)
+
+
+def cpu_all_cores(items, args):
+    """The same sample split into row ranges over independent oracle processes,
+    one per host core (at most MAX_ORACLE_PROCS), started with spawn: wall-clock
+    throughput of the oracle as it stands on the whole host."""
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    procs = max(1, min(cores, MAX_ORACLE_PROCS))
+    parts = [[] for _ in range(procs)]
+    for label, xb, fmt, block, rot, gmode in items:
+        rows = xb.shape[0]
+        for q in range(procs):
+            lo, hi = rows * q // procs, rows * (q + 1) // procs
+            if hi > lo:
+                parts[q].append((label, xb[lo:hi].copy(), fmt, block, rot, gmode))
+    payloads = [(part, args.search, args.outlier_stats) for part in parts]
+    # every wait is bounded: a pool whose workers cannot start (for instance when
+    # __main__ cannot be re-imported by spawn) raises here instead of hanging
+    with mp.get_context("spawn").Pool(procs, initializer=_oracle_init) as pool:
+        pool.map_async(_oracle_worker, [([], None, None)] * procs, chunksize=1).get(timeout=120)
+        t0 = time.perf_counter()
+        n = sum(pool.map_async(_oracle_worker, payloads, chunksize=1).get(timeout=120 + 20 * args.cpu_seconds))
+        dt = time.perf_counter() - t0
+    return {"value": n / dt / 1e9, "unit": "Gelem/s", "cores": procs, "host_cores": cores,
+            "sample": f"the same {n} elements in {procs} row ranges, one oracle process each, {dt:.2f} s wall"}
+
+
 def cpu_baseline(name, args):
-    """Oracle throughput on ~args.cpu_seconds of single-threaded CPU work."""
+    """Oracle throughput on ~args.cpu_seconds of single-threaded CPU work, and
+    the same sample over all host cores in independent processes."""
     probe = cpu_sample_items(name, args, 1_000_000)
     t0 = time.perf_counter()
     n = oracle_sample_step(probe, args.search, args.outlier_stats)
@@ -406,9 +446,14 @@ def cpu_baseline(name, args):
     t0 = time.perf_counter()
     n = oracle_sample_step(items, args.search, args.outlier_stats)
     dt = time.perf_counter() - t0
-    return {"value": n / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} elements: the first rows of each of the {len(items)} tensors, same recipe, "
-                      f"drawn on the host; quantize + dequantize + block MSE, single-threaded C, {dt:.1f} s"}
+    out = {"value": n / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+           "sample": f"{n} elements: the first rows of each of the {len(items)} tensors, same recipe, "
+                     f"drawn on the host; quantize + dequantize + block MSE, single-threaded C, {dt:.1f} s"}
+    try:
+        out["all_cores"] = cpu_all_cores(items, args)
+    except Exception as e:                      # reported, never fatal to the GPU measurement
+        out["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"}
+    return out
 
 
 # --------------------------------------------------------------------------- reference arm

@@ -42,3 +42,12 @@ def test_reference_arm_line(extra, capsys, monkeypatch):
         assert "MSE search" in line["config"]["block_scales"]
     if "--outlier-stats" in extra:
         assert "P99.9" in line["config"]["outlier_stats"]
+
+
+def test_cpu_baseline_single_core_and_all_cores():
+    args = bench.parse_args(["--cpu-seconds", "0.3"])
+    cb = bench.cpu_baseline("nvfp4_qwen25_7b_mlp", args)
+    assert cb["cores"] == 1 and cb["kind"] == "oracle" and cb["value"] > 0
+    ac = cb["all_cores"]
+    assert "unavailable" not in ac, ac
+    assert ac["value"] > 0 and 1 <= ac["cores"] <= bench.MAX_ORACLE_PROCS
