@@ -168,6 +168,8 @@ def fp4q_quantize_search(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="
         raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
     if gscale is None and gmode != FP4Q_GLOBAL_NONE:
         gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    if gmode == FP4Q_GLOBAL_FROM_AMAX and gscale.numel() < 2:
+        raise ValueError("from_amax mode needs gscale with 2 floats: [amax in, G out]")
     _need_cuda(codes, scales, gscale)
     st = lib().fp4q_quantize_search(_ptr(x), rows, cols, fmt, block, rot, gmode, below, above, _ptr(codes),
                                     _ptr(scales), _ptr(gscale), _stream(stream))
