@@ -392,11 +392,11 @@ int orc_quantize_f32(const float* x, int64_t rows, int64_t cols, int fmt, int bl
 /* (codes outside the format's finite range are skipped); a candidate         */
 /* replaces the best so far only when its error is strictly smaller, so ties  */
 /* keep the earlier one and the max rule wins any tie.  The error of a scale  */
-/* S is sum_i (y_i - v_i)^2 with v_i = fp32(decode(E2M1(y_i / S)) S), and     */
-/* v_i = 0 when S = 0 (a zero-rounded block).  The pages fix no precision for */
-/* this choice, so it is taken in fp32, as the GPU kernel takes it: each term */
-/* d_i = fp32(y_i - v_i) is added as acc = fma(d_i, d_i, acc), in element     */
-/* order (the kernel's order differs; its tests allow for that).              */
+/* S is sum_i (y_i - v_i)^2 with v_i = fp32(decode(E2M1(y_i / S)) S), and    */
+/* v_i = 0 when S = 0 (a zero-rounded block).  The pages fix no precision, so */
+/* the criterion is the exact error: each d_i = y_i - v_i is exact in fp64,   */
+/* its square is exact (24-bit significands), and the fp64 sum of b <= 256    */
+/* such terms is within 2^-45 relative of the true sum.                       */
 
 static int last_finite_code(int fmt)
 {
@@ -405,16 +405,16 @@ static int last_finite_code(int fmt)
     return 0xfe;
 }
 
-static float block_sq_error(const float* y, int block, float S)
+static double block_sq_error(const float* y, int block, float S)
 {
-    float acc = 0.0f;
+    double sum = 0.0;
     for (int i = 0; i < block; ++i) {
         float v = 0.0f;
         if (S != 0.0f) v = (float)((double)orc_e2m1_decode(orc_e2m1_encode(y[i] / S)) * (double)S);
-        float d = y[i] - v;
-        acc = fmaf(d, d, acc);
+        double d = (double)y[i] - (double)v;
+        sum += d * d;
     }
-    return acc;
+    return sum;
 }
 
 int orc_quantize_search_f32(const float* x, int64_t rows, int64_t cols, int fmt, int block,
@@ -435,11 +435,11 @@ int orc_quantize_search_f32(const float* x, int64_t rows, int64_t cols, int fmt,
     for (int64_t b0 = 0, bi = 0; b0 < n; b0 += block, ++bi) {
         const int s0 = scales[bi];
         int best = s0;
-        float best_err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)s0, G));
+        double best_err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)s0, G));
         for (int j = 1; j <= above + below; ++j) {
             const int c = j <= above ? s0 + j : s0 - (j - above);
             if (c < 0 || c > last) continue;
-            float err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)c, G));
+            double err = block_sq_error(y + b0, block, scale_of_code(fmt, (uint8_t)c, G));
             if (err < best_err) {
                 best = c;
                 best_err = err;

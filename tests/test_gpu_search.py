@@ -1,11 +1,13 @@
 """Parity of fp4q_quantize_search (MSE-optimised block scales, "Bridging the
 Gap", s3, MR-GPTQ item 2) with the oracle, through the C ABI.
 
-Both sides decide each block in fp32, but sum a block's squared errors in
-different orders (the kernel in two interleaved running sums, the oracle in
-element order), so their choice may differ only between two codes whose errors
-agree to fp32 rounding: |E1 - E2| <= 2 (b + 4) 2^-24 max(E1, E2), with E the
-fp64 errors the oracle measures for each choice.  Everything else is unique:
+The oracle decides each block on the exact squared error (an fp64 sum of
+fp64 squared differences); the kernel decides on fp32 sums (two interleaved
+running sums of fused multiply-adds).  Each fp32 sum of b non-negative rounded
+terms is within (b + 4) 2^-24 relative of the exact one, so the two choices may
+differ only between two codes whose exact errors agree to that rounding:
+|E1 - E2| <= 2 (b + 4) 2^-24 max(E1, E2), with E the fp64 errors the oracle
+measures for each choice.  Everything else is unique:
  * unrotated: the chosen scale lies in the window around the max-rule code,
    and the codes are bit-exact against the oracle's quantizer for the GPU's
    scale bytes; where the scale bytes agree they are simply equal;
