@@ -87,20 +87,39 @@ def test_nvfp4_qwen25_7b_mlp_full(fq):
                 assert abs(t[i] - o_terms[i]) <= 2e-6 * o_terms[0]
 
 
+def _check_whole_rotated(x, codes, scales, gs, fmt, block, rot, gmode):
+    """The whole tensor against the oracle's own run, per-tensor scale included:
+    G (COMPUTE mode) from the oracle's fp64 rotation of every element, then
+    every scale byte and every code under the rotated-path rule."""
+    xh = bf16_bits(x)
+    o_codes, o_scales, o_G = oracle.quantize(xh, fmt, block, rot, gmode)
+    g = {"codes": codes.cpu().numpy(), "scales": scales.cpu().numpy(),
+         "G": float(gs.item()) if gs is not None else 1.0}
+    return check_rotated(g, {"codes": o_codes, "scales": o_scales, "G": o_G},
+                         oracle.bf16_bits_to_f32(xh), fmt, block, rot)
+
+
 def test_rotated_activations_full_8192x5120(fq):
+    """Every rotation size with MXFP4 (sampled rows against the oracle) and
+    NVFP4 with a computed per-tensor scale (the whole tensor against the
+    oracle's own run, so the rotated G is the oracle's, not the GPU's)."""
     x, _ = workloads.student_t_outliers_bf16(8192, 5120, seed=77, device="cuda")
     for rot in workloads.ACT_ROTATIONS:
         for fmt, block, gmode in [(E8, 32, NONE), (U4, 16, COMP)]:
             codes, scales, gs, bm, terms = _run_full(fq, x, fmt, block, rot, gmode)
             torch.cuda.synchronize()
-            G = 1.0
             if gmode == COMP:
-                G = float(gs.item())     # checked against the oracle's own G on sampled rows below
                 xf = oracle.bf16_bits_to_f32(bf16_bits(x))
                 if rot == 0:
-                    assert np.float32(G) == np.float32(oracle.global_scale_from_amax(oracle.tensor_amax(xf)))
-            _check_sampled(fq, x, codes, scales, gs, bm, fmt, block, rot, gmode, G,
-                           _sample_rows(8192, 12, rot + block))
+                    assert np.float32(gs.item()) == np.float32(
+                        oracle.global_scale_from_amax(oracle.tensor_amax(xf)))
+                    _check_sampled(fq, x, codes, scales, gs, bm, fmt, block, rot, gmode, float(gs.item()),
+                                   _sample_rows(8192, 12, rot + block))
+                else:
+                    _check_whole_rotated(x, codes, scales, gs, fmt, block, rot, gmode)
+            else:
+                _check_sampled(fq, x, codes, scales, gs, bm, fmt, block, rot, gmode, 1.0,
+                               _sample_rows(8192, 12, rot + block))
             _terms_consistent(bm, terms)
 
 
@@ -108,8 +127,10 @@ def test_qwen25_14b_weight_pass(fq):
     """48 layers x {q, k, v, o, gate, up, down}, sigma_l = 0.02 * U(0.5, 1.5);
     MXFP4 and NVFP4 (per-tensor scale), without and with a 32-wide rotation.
     Sampled rows of every layer's first tensor (and of every tensor of every
-    sixth layer) against the oracle; the whole k projection of every fourth
-    layer against the oracle's MSE terms; every layer's split against the
+    sixth layer) against the oracle, quantized with the GPU's G; the whole k
+    projection of every fourth layer against the oracle's MSE terms and, with
+    the rotation, against the oracle's own whole run (its own rotated G, every
+    scale byte and code); every layer's split against the
     Gaussian model as a sanity bound (bf16 rounding of the inputs moves block
     maxima onto the power-of-two and scale-code boundaries where the
     max-element error jumps, so the continuous model is only good to ~1-2%
@@ -138,6 +159,9 @@ def test_qwen25_14b_weight_pass(fq):
                 if check:
                     _check_sampled(fq, x, codes, scales, gs, bm, fmt, block, rot, gmode, G,
                                    _sample_rows(t.rows, 2, layer * 7 + ti))
+                if whole and rot:
+                    # the rotated per-tensor scale and every code against the oracle's own whole run
+                    _check_whole_rotated(x, codes, scales, gs, fmt, block, rot, gmode)
                 if whole and (rot == 0 or layer % 12 == 0):
                     _, o_terms = oracle.block_mse(xh, codes.cpu().numpy(), scales.cpu().numpy(), G, fmt,
                                                   block, rot)
