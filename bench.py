@@ -2,14 +2,20 @@
 """Benchmark of the block-wise microscaling FP4 hot path on B200.
 
 One step = the whole hot path over one batch of synthetic input: for every
-tensor of the workload, the per-tensor amax, the per-tensor scale, the fused
-(rotate+)scale+round+pack quantize kernel that also measures the per-block /
-per-tensor MSE with its three-term split, and dequantization.  Default workload: NVFP4 (block 16,
-UE4M3 block scales, FP32 per-tensor scale amax/(6*448)) on the nine Qwen2.5-7B
-MLP weights gate/up 18944x3584 and down 3584x18944 at sigma 0.005/0.02/0.05
-(611M elements, 1.22 GB of bf16 per step: larger than L2).
+tensor of the workload, the per-tensor amax (NVFP4 with a computed per-tensor
+scale), and the fused (rotate+)scale+round+pack quantize kernel that also
+measures the per-block / per-tensor MSE with its three-term split and writes
+the dequantized tensor.
+
+Default workload: the whole-model weight pass at Qwen2.5-14B shapes, 48 layers
+x {q 5120x5120, k/v 1024x5120, o 5120x5120, gate/up 13824x5120, down
+5120x13824} bf16, N(0, sigma_l^2) with sigma_l = 0.02 U(0.5, 1.5) per layer,
+in four variants: MXFP4 (block 32, E8M0) and NVFP4 (block 16, UE4M3 under an
+FP32 per-tensor scale), each without and with the 32-wide Hadamard rotation
+(13.2 G elements and 26.4 GB of bf16 per variant, 52.8 G elements per step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp4q|reference]
+                    [--workload NAME]
 
 Prints one JSON line (rank 0).  Under torchrun each rank processes its own
 copy of the workload (independent tensors, no data-path collective): weak
@@ -36,15 +42,28 @@ E8, U4, U5 = 0, 1, 2
 NONE, COMP, GIVEN, FROM_AMAX = 0, 1, 2, 3
 
 
+# Timed and warm-up steps per workload when not given: about ten seconds of
+# timed device work each.
+WORKLOAD_DEFAULTS = {
+    "qwen25_14b_weight_pass": dict(steps=100, warmup=3, e2e_steps=2),
+    "nvfp4_qwen25_7b_mlp": dict(steps=200, warmup=10, e2e_steps=10),
+    "rotated_activations_8192x5120": dict(steps=200, warmup=10, e2e_steps=10),
+    "block_size_sweep_4096": dict(steps=100, warmup=5, e2e_steps=5),
+    "mxfp4_gaussian_1024x1024": dict(steps=200, warmup=10, e2e_steps=10),
+}
+# The four variants of the whole-model weight pass: (name, fmt, block, rot, gmode).
+WEIGHT_PASS_VARIANTS = (("mxfp4_rot0", 0, 32, 0, 0), ("nvfp4_rot0", 1, 16, 0, 1),
+                        ("mxfp4_rot32", 0, 32, 32, 0), ("nvfp4_rot32", 1, 16, 32, 1))
+
+
 # --------------------------------------------------------------------------- args / dist
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: per workload)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: per workload)")
     ap.add_argument("--impl", choices=["fp4q", "reference"], default="fp4q")
-    ap.add_argument("--workload", default="nvfp4_qwen25_7b_mlp",
-                    choices=["nvfp4_qwen25_7b_mlp", "rotated_activations_8192x5120", "mxfp4_gaussian_1024x1024"])
+    ap.add_argument("--workload", default="qwen25_14b_weight_pass", choices=list(WORKLOAD_DEFAULTS))
     ap.add_argument("--rot", type=int, default=128, help="rotation for the activation workload")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"], help="format for the activation workload")
     ap.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: max(3, steps // 20))")
@@ -61,6 +80,11 @@ def parse_args(argv=None):
                     help="add the activation outlier statistics (max, nearest-rank P-quantile of |x|, channel "
                          "maxima: fp4q_outlier_stats) to every tensor of the step")
     args = ap.parse_args(argv)
+    d = WORKLOAD_DEFAULTS[args.workload]
+    if args.steps is None:
+        args.steps = d["steps"]
+    if args.warmup is None:
+        args.warmup = d["warmup"]
     args.search = None
     if args.scale_search:
         below, above = (int(v) for v in args.scale_search.split(","))
@@ -103,11 +127,45 @@ def rank_seed(base: int, rank: int) -> int:
 
 
 # --------------------------------------------------------------------------- workload
+def item_tag(label: str) -> str:
+    """Variant of a workload item ("nvfp4_rot32" in "nvfp4_rot32/L7.q"), or ""."""
+    return label.split("/", 1)[0] if "/" in label else ""
+
+
+def weight_pass_items(xs, per_layer: int):
+    """Items and launch groups of the whole-model weight pass over the tensors
+    xs = [(name, x)] (layer-major, per_layer tensors a layer): variant by
+    variant, layer by layer; within a layer group a step runs the layer's amax
+    passes, then its quantizer passes, so that a layer's 550 MB are read between
+    a tensor's amax and its quantizer and both read HBM."""
+    out, groups = [], []
+    for vname, fmt, block, rot, gmode in WEIGHT_PASS_VARIANTS:
+        for l0 in range(0, len(xs), per_layer):
+            groups.append(list(range(len(out), len(out) + len(xs[l0:l0 + per_layer]))))
+            for lbl, x in xs[l0:l0 + per_layer]:
+                out.append((f"{vname}/{lbl}", x, fmt, block, rot, gmode))
+    return out, groups
+
+
 def build_workload(name: str, device, rank: int, args):
-    """[(label, x bf16 [rows, cols], fmt, block, rot, gmode)] on `device`."""
+    """([(label, x bf16 [rows, cols], fmt, block, rot, gmode)], groups) on `device`.
+
+    groups: lists of item indices; a step runs, group by group, the first call
+    of every item of the group, then the second call of every item, and so on.
+    """
     import workloads as W
-    out = []
-    if name == "nvfp4_qwen25_7b_mlp":
+    out, groups = [], None
+    if name == "qwen25_14b_weight_pass":
+        # one bf16 copy of the 48 x 7 weights (26.4 GB); the four variants read it in
+        # turn, variant by variant, so each pass streams the whole model from HBM
+        sigmas = W.layer_sigmas(W.QWEN25_14B_LAYERS, 0.02, 0.5, rank_seed(14, rank))
+        xs = []
+        for layer, sigma in enumerate(sigmas):
+            for ti, t in enumerate(W.QWEN25_14B_LAYER):
+                xs.append((f"L{layer}.{t.name}",
+                           W.gaussian_bf16(t.rows, t.cols, sigma, rank_seed(100000 + 16 * layer + ti, rank), device)))
+        out, groups = weight_pass_items(xs, len(W.QWEN25_14B_LAYER))
+    elif name == "nvfp4_qwen25_7b_mlp":
         for si, sigma in enumerate(W.QWEN25_7B_SIGMAS):
             for ti, t in enumerate(W.QWEN25_7B_MLP):
                 x = W.gaussian_bf16(t.rows, t.cols, sigma, rank_seed(1000 + 10 * si + ti, rank), device)
@@ -116,10 +174,21 @@ def build_workload(name: str, device, rank: int, args):
         x, _ = W.student_t_outliers_bf16(8192, 5120, rank_seed(77, rank), device=device)
         fmt, block = (U4, 16) if args.fmt == "nvfp4" else (E8, 32)
         out.append((f"act_rot{args.rot}", x, fmt, block, args.rot, COMP if fmt == U4 else NONE))
+    elif name == "block_size_sweep_4096":
+        # UE4M3 without a per-tensor scale (the sweep), E8M0, UE4M3 under a per-tensor
+        # scale and UE5M3, every block size, on four 4096 x 4096 tensors (33.5 MB each)
+        xs = [W.gaussian_bf16(4096, 4096, sg, rank_seed(300 + si, rank), device)
+              for si, sg in enumerate(W.SWEEP_SIGMAS)]
+        for tag, fmt, gmode in (("ue4m3", U4, NONE), ("e8m0", E8, NONE), ("ue4m3s", U4, COMP), ("ue5m3", U5, NONE)):
+            for block in W.SWEEP_BLOCKS:
+                for si, x in enumerate(xs):
+                    out.append((f"{tag}_b{block}/s{W.SWEEP_SIGMAS[si]}", x, fmt, block, 0, gmode))
     else:
         x = W.gaussian_bf16(1024, 1024, 0.02, rank_seed(0, rank), device)
         out.append(("w1024", x, E8, 32, 0, NONE))
-    return out
+    if groups is None:
+        groups = [[i] for i in range(len(out))]
+    return out, groups
 
 
 def bytes_per_element(block: int):
@@ -136,6 +205,21 @@ def bytes_per_element(block: int):
     }
 
 
+def stage_kind(stage: str) -> str:
+    """Kernel of a stage name ("quantize_mse_dequantize" in "quantize_mse_dequantize@nvfp4_rot32")."""
+    return stage.split("@", 1)[0]
+
+
+def launches_of(stage: str, n: int) -> int:
+    """Kernel launches one C-ABI call of `stage` makes on n elements.  The outlier
+    statistics: one histogram pass and a scan below 2^22 elements; above, a
+    sampled pass, the threshold scan, the main pass, a scan, and a pass and a
+    scan that return at once unless the threshold missed."""
+    if stage_kind(stage) == "outlier_stats":
+        return 6 if n >= (1 << 22) else 2
+    return 1
+
+
 class Pipeline:
     """Device buffers and the per-step launch sequence for a workload.
 
@@ -145,9 +229,8 @@ class Pipeline:
     one kernel is the event before the next.
     """
 
-
     def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False, search=None,
-                 outlier_p=None):
+                 outlier_p=None, groups=None):
         import torch
         self.fq, self.items, self.device = fq, items, device
         L = fq.lib()
@@ -157,13 +240,18 @@ class Pipeline:
         self.gs_all = torch.zeros((len(items), 2), dtype=torch.float32, device=device)
         self.any_comp = any(gm == COMP for *_, gm in items)
         separate_mse = separate_mse or search is not None     # the search has no fused MSE pass
+        deq_of = {}                # one dequantized-output buffer per input tensor, shared by its variants
         for ti, (label, x, fmt, block, rot, gmode) in enumerate(items):
             rows, cols = x.shape
+            tag = item_tag(label)
+            sfx = f"@{tag}" if tag else ""
+            if x.data_ptr() not in deq_of:
+                deq_of[x.data_ptr()] = torch.empty((rows, cols), dtype=torch.bfloat16, device=device)
             b = dict(
                 codes=torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
                 scales=torch.empty((rows, cols // block), dtype=torch.uint8, device=device),
                 gscale=self.gs_all[ti],                                            # [amax, G]
-                deq=torch.empty((rows, cols), dtype=torch.bfloat16, device=device),
+                deq=deq_of[x.data_ptr()],
                 bm=torch.empty((rows, cols // block), dtype=torch.float32, device=device),
                 terms=torch.empty((4,), dtype=torch.float64, device=device),
                 ws=torch.zeros((fq.fp4q_block_mse_workspace_size(rows, cols, block),), dtype=torch.uint8,
@@ -183,64 +271,72 @@ class Pipeline:
             g = p["gscale"] + 4 if comp else None
             seq = []
             if outlier_p is not None:
-                seq.append(("outlier_stats", L.fp4q_outlier_stats, (x.data_ptr(), rows, cols, float(outlier_p),
-                                                                    p["ostats"], p["ocols"], p["ows"],
-                                                                    b["ows"].numel(), sh)))
+                seq.append(("outlier_stats" + sfx, L.fp4q_outlier_stats,
+                            (x.data_ptr(), rows, cols, float(outlier_p), p["ostats"], p["ocols"], p["ows"],
+                             b["ows"].numel(), sh)))
             if comp:
-                seq.append(("amax", L.fp4q_tensor_amax_accumulate, (x.data_ptr(), rows, cols, rot, p["gscale"], sh)))
+                seq.append(("amax" + sfx, L.fp4q_tensor_amax_accumulate,
+                            (x.data_ptr(), rows, cols, rot, p["gscale"], sh)))
             gm = FROM_AMAX if comp else NONE
             if search is not None:
-                seq.append(("quantize_search", L.fp4q_quantize_search,
+                seq.append(("quantize_search" + sfx, L.fp4q_quantize_search,
                             (x.data_ptr(), rows, cols, fmt, block, rot, gm, search[0], search[1], p["codes"],
                              p["scales"], gq, sh)))
-                seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
-                                                            fmt, block, rot, p["bm"], p["terms"], p["ws"],
-                                                            b["ws"].numel(), sh)))
+                seq.append(("block_mse" + sfx, L.fp4q_block_mse,
+                            (x.data_ptr(), p["codes"], p["scales"], g, rows, cols, fmt, block, rot, p["bm"],
+                             p["terms"], p["ws"], b["ws"].numel(), sh)))
             elif separate_mse:
-                seq.append(("quantize", L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot, gm,
-                                                          p["codes"], p["scales"], gq, sh)))
-                seq.append(("block_mse", L.fp4q_block_mse, (x.data_ptr(), p["codes"], p["scales"], g, rows, cols,
-                                                            fmt, block, rot, p["bm"], p["terms"], p["ws"],
-                                                            b["ws"].numel(), sh)))
+                seq.append(("quantize" + sfx, L.fp4q_quantize, (x.data_ptr(), rows, cols, fmt, block, rot, gm,
+                                                                p["codes"], p["scales"], gq, sh)))
+                seq.append(("block_mse" + sfx, L.fp4q_block_mse,
+                            (x.data_ptr(), p["codes"], p["scales"], g, rows, cols, fmt, block, rot, p["bm"],
+                             p["terms"], p["ws"], b["ws"].numel(), sh)))
             elif separate_dequant:
-                seq.append(("quantize_mse", L.fp4q_quantize_mse,
+                seq.append(("quantize_mse" + sfx, L.fp4q_quantize_mse,
                             (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], gq, p["bm"],
                              p["terms"], p["ws"], b["ws"].numel(), sh)))
             else:
                 # quantize, the MSE split and the dequantized bf16 tensor in one pass over x
-                seq.append(("quantize_mse_dequantize", L.fp4q_quantize_mse_dequantize,
+                seq.append(("quantize_mse_dequantize" + sfx, L.fp4q_quantize_mse_dequantize,
                             (x.data_ptr(), rows, cols, fmt, block, rot, gm, p["codes"], p["scales"], gq, p["deq"],
                              p["bm"], p["terms"], p["ws"], b["ws"].numel(), sh)))
             if separate_mse or separate_dequant:
-                seq.append(("dequantize", L.fp4q_dequantize, (p["codes"], p["scales"], g, rows, cols, fmt, block, 0,
-                                                              0, p["deq"], sh)))
+                seq.append(("dequantize" + sfx, L.fp4q_dequantize,
+                            (p["codes"], p["scales"], g, rows, cols, fmt, block, 0, 0, p["deq"], sh)))
             self.calls.append(seq)
+        # launch order: group by group, the j-th call of every item of the group
+        groups = groups if groups is not None else [[i] for i in range(len(items))]
+        self.order = []
+        for grp in groups:
+            for j in range(max(len(self.calls[i]) for i in grp)):
+                self.order.extend((i, j) for i in grp if j < len(self.calls[i]))
+        assert sorted(self.order) == sorted((i, j) for i in range(len(items)) for j in range(len(self.calls[i])))
         self.elements = sum(x.numel() for _, x, *_ in items)
-        # kernels per step: amax (per-tensor scale), quantize (+MSE, reduced in-kernel, + dequantized output),
-        # [block MSE], [dequantize]
-        # outlier statistics: one histogram pass and a scan below 2^22 elements; above, a sampled
-        # pass, the threshold scan, the main pass, a scan, and a pass and a scan that return at once
-        # unless the threshold missed
-        self.launches_per_step = sum(1 + (1 if gm == COMP else 0) + (2 if separate_mse else 0)
-                                     + (1 if separate_dequant and not separate_mse else 0)
-                                     + (0 if outlier_p is None else (6 if x.numel() >= (1 << 22) else 2))
-                                     for _, x, *_, gm in items)
-        self.events_per_step = 1 + sum(len(seq) for seq in self.calls)
+        self.launches_per_step = sum(launches_of(self.calls[i][j][0], items[i][1].numel()) for i, j in self.order)
+        self.events_per_step = 1 + len(self.order)
 
     def step(self, stream, ev=None):
         """Enqueue one step; ev = events_per_step timing events or None."""
         bad = 0
-        j = 0
-        if ev is not None:
-            ev[0].record(stream)
         if self.any_comp:
             self.gs_all.zero_()       # the maxima accumulate from 0
-        for seq in self.calls:
-            for stage, fn, args in seq:
-                bad |= fn(*args)
-                if ev is not None:
-                    j += 1
-                    ev[j].record(stream)
+        if ev is not None:
+            ev[0].record(stream)
+        for j, (i, k) in enumerate(self.order):
+            _, fn, args = self.calls[i][k]
+            bad |= fn(*args)
+            if ev is not None:
+                ev[j + 1].record(stream)
+        if bad:
+            raise RuntimeError(f"a C-ABI call returned an error status ({bad})")
+
+    def run_items(self, idx):
+        """Enqueue every call of the items idx, in step order (end-to-end pass)."""
+        sel = set(idx)
+        bad = 0
+        for i, k in self.order:
+            if i in sel:
+                bad |= self.calls[i][k][1](*self.calls[i][k][2])
         if bad:
             raise RuntimeError(f"a C-ABI call returned an error status ({bad})")
 
@@ -249,13 +345,8 @@ class Pipeline:
         return [torch.cuda.Event(enable_timing=True) for _ in range(self.events_per_step)]
 
     def stage_times(self, ev):
-        """[(tensor index, stage, ms)] of one step's events."""
-        out, j = [], 0
-        for i, seq in enumerate(self.calls):
-            for stage, _, _ in seq:
-                out.append((i, stage, ev[j].elapsed_time(ev[j + 1])))
-                j += 1
-        return out
+        """[(item index, stage, ms)] of one step's events."""
+        return [(i, self.calls[i][k][0], ev[j].elapsed_time(ev[j + 1])) for j, (i, k) in enumerate(self.order)]
 
 
 # --------------------------------------------------------------------------- clocks
@@ -376,7 +467,28 @@ def cpu_sample_items(name: str, args, elements_target: int):
     import torch
     import workloads as W
     out = []
-    if name == "nvfp4_qwen25_7b_mlp":
+    if name == "qwen25_14b_weight_pass":
+        # the first rows of the seven tensors of layers 0, 16, 32 and 47, each in the four variants
+        layers = (0, 16, 32, 47)
+        sigmas = W.layer_sigmas(W.QWEN25_14B_LAYERS, 0.02, 0.5, 14)
+        per = max(1, elements_target // (len(layers) * len(W.QWEN25_14B_LAYER) * len(WEIGHT_PASS_VARIANTS)))
+        for vname, fmt, block, rot, gmode in WEIGHT_PASS_VARIANTS:
+            for layer in layers:
+                for ti, t in enumerate(W.QWEN25_14B_LAYER):
+                    rows = max(1, min(t.rows, per // t.cols))
+                    x = W.gaussian_bf16(rows, t.cols, sigmas[layer], 100000 + 16 * layer + ti)
+                    out.append((f"{vname}/L{layer}.{t.name}", x.view(torch.int16).numpy().view(np.uint16), fmt,
+                                block, rot, gmode))
+    elif name == "block_size_sweep_4096":
+        per = max(1, elements_target // (4 * len(W.SWEEP_BLOCKS) * len(W.SWEEP_SIGMAS)))
+        rows = max(1, min(4096, per // 4096))
+        xs = [W.gaussian_bf16(rows, 4096, sg, 300 + si) for si, sg in enumerate(W.SWEEP_SIGMAS)]
+        for tag, fmt, gmode in (("ue4m3", U4, NONE), ("e8m0", E8, NONE), ("ue4m3s", U4, COMP), ("ue5m3", U5, NONE)):
+            for block in W.SWEEP_BLOCKS:
+                for si, x in enumerate(xs):
+                    out.append((f"{tag}_b{block}/s{W.SWEEP_SIGMAS[si]}", x.view(torch.int16).numpy().view(np.uint16),
+                                fmt, block, 0, gmode))
+    elif name == "nvfp4_qwen25_7b_mlp":
         per = max(1, elements_target // 9)
         for si, sigma in enumerate(W.QWEN25_7B_SIGMAS):
             for ti, t in enumerate(W.QWEN25_7B_MLP):
@@ -447,7 +559,7 @@ def cpu_baseline(name, args):
     n = oracle_sample_step(items, args.search, args.outlier_stats)
     dt = time.perf_counter() - t0
     out = {"value": n / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-           "sample": f"{n} elements: the first rows of each of the {len(items)} tensors, same recipe, "
+           "sample": f"{n} elements: {sample_note(name)} ({len(items)} tensor runs), same recipe, "
                      f"drawn on the host; quantize + dequantize + block MSE, single-threaded C, {dt:.1f} s"}
     try:
         out["all_cores"] = cpu_all_cores(items, args)
@@ -462,7 +574,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     import numpy as np
-    per_step = 6_000_000 if args.workload == "nvfp4_qwen25_7b_mlp" else 2_000_000
+    per_step = {"nvfp4_qwen25_7b_mlp": 6_000_000, "qwen25_14b_weight_pass": 3_000_000,
+                "block_size_sweep_4096": 6_000_000}.get(args.workload, 2_000_000)
     items = cpu_sample_items(args.workload, args, per_step)
     for _ in range(args.warmup):
         oracle_sample_step(items, args.search, args.outlier_stats)
@@ -483,13 +596,33 @@ def run_reference(args):
                                         f"max, P{100 * args.outlier_stats:g} of |x| and channel maxima per tensor",
                        "note": "the CPU oracle (single-threaded C) on a bounded sample of the workload"},
             "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{n // args.steps} elements per step: the first rows of every tensor"},
+                             "sample": f"{n // args.steps} elements per step: {sample_note(args.workload)}"},
             "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
 
 
 # --------------------------------------------------------------------------- main (CUDA path)
+def sample_note(name: str) -> str:
+    if name == "qwen25_14b_weight_pass":
+        return ("the first rows of the seven tensors of layers 0, 16, 32 and 47 in each of the four variants "
+                "(a layer subset; the throughput extrapolates to the 48-layer pass, every tensor being "
+                "processed at the same per-element cost)")
+    if name == "block_size_sweep_4096":
+        return "the first rows of the four sigma tensors, every block size and scale format"
+    return "the first rows of every tensor"
+
+
+def describe_format(items):
+    names = {U4: "NVFP4 UE4M3", E8: "MXFP4 E8M0", U5: "UE5M3"}
+    seen = []
+    for label, x, fmt, block, rot, gmode in items:
+        d = f"{names[fmt]} b{block}" + (" + FP32 per-tensor scale" if gmode == COMP else "") + f", rot {rot}"
+        if d not in seen:
+            seen.append(d)
+    return seen if len(seen) > 1 else seen[0]
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -505,12 +638,14 @@ def main(argv=None):
     init_dist(world, "nccl", device)
     import torch.distributed as dist
 
-    items = build_workload(args.workload, device, rank, args)
+    items, groups = build_workload(args.workload, device, rank, args)
     stream = torch.cuda.Stream(device)
     stream.wait_stream(torch.cuda.current_stream())
     pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse,
-                    separate_dequant=args.separate_dequant, search=args.search, outlier_p=args.outlier_stats)
-    in_l2 = sum(x.numel() * 2 for _, x, *_ in items) < 256 * 2 ** 20
+                    separate_dequant=args.separate_dequant, search=args.search, outlier_p=args.outlier_stats,
+                    groups=groups)
+    distinct_bytes = sum(x.numel() * 2 for x in {x.data_ptr(): x for _, x, *_ in items}.values())
+    in_l2 = distinct_bytes < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
 
     with torch.cuda.stream(stream):
@@ -528,6 +663,7 @@ def main(argv=None):
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
+    kernel_steps = max(1, min(args.steps, max(3, 20000 // pipe.events_per_step)))
     with sampler, torch.cuda.stream(stream):
         for k in range(args.steps):
             bounds[k][0].record(stream)
@@ -541,17 +677,17 @@ def main(argv=None):
         local_ms = sum(a.elapsed_time(b) for a, b in bounds)
         total_ms = reduce_max(local_ms, device)
 
-        # ---- per-kernel pass (the same K steps, an event after every C-ABI call on the
-        # launching stream): kernel shares and the dominant kernel's achieved bandwidth
-        events = [pipe.new_events() for _ in range(args.steps)]
-        for k in range(args.steps):
+        # ---- per-kernel pass (kernel_steps more steps, an event after every C-ABI call
+        # on the launching stream): kernel shares and the dominant kernel's achieved bandwidth
+        events = [pipe.new_events() for _ in range(kernel_steps)]
+        for k in range(kernel_steps):
             pipe.step(stream, events[k])
             if flush is not None:
                 flush.zero_()
         torch.cuda.synchronize()
 
     per_kernel = {}
-    for k in range(args.steps):
+    for k in range(kernel_steps):
         for i, stage, ms in pipe.stage_times(events[k]):
             per_kernel.setdefault(stage, []).append((i, ms))
     elements_step = pipe.elements
@@ -563,12 +699,16 @@ def main(argv=None):
     step_bytes = 0.0
     for stage, lst in per_kernel.items():
         tot_ms = sum(t for _, t in lst)
-        byts = 0.0
+        byts = elems = 0.0
         for i, t in lst:
             _, x, fmt, block, rot, gmode = items[i]
-            byts += bytes_per_element(block).get(stage, 0.0) * x.numel()
-        step_bytes += byts / args.steps
-        kernels[stage] = {"ms_per_step": tot_ms / args.steps, "share": None,
+            byts += bytes_per_element(block).get(stage_kind(stage), 0.0) * x.numel()
+            elems += x.numel()
+        step_bytes += byts / kernel_steps
+        kernels[stage] = {"ms_per_step": tot_ms / kernel_steps, "share": None,
+                          "launches_per_step": len(lst) / kernel_steps,
+                          "elements_per_launch": elems / len(lst),
+                          "algorithmic_bytes_per_launch": byts / len(lst),
                           "GB_per_s": (byts / 1e9) / (tot_ms / 1e3) if tot_ms > 0 else None}
     busy = sum(v["ms_per_step"] for v in kernels.values())
     for v in kernels.values():
@@ -576,15 +716,12 @@ def main(argv=None):
         v["frac_of_peak"] = (v["GB_per_s"] / peak) if v["GB_per_s"] else None
     dominant = max(kernels, key=lambda s: kernels[s]["ms_per_step"])
     dk = kernels[dominant]
-    launches = sum(1 for _ in per_kernel[dominant]) / args.steps
-    _, x0, _, block0, _, _ = items[0]
-    dom_bpe = bytes_per_element(block0).get(dominant, 0.0)
     tpe = ncu_traffic(dominant, args.workload)
-    per_launch_elems = elements_step / max(launches, 1)
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": dk["GB_per_s"], "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": dk["GB_per_s"] / peak,
-                "traffic": (tpe * per_launch_elems if tpe is not None else None),
-                "algorithmic_bytes_per_launch": dom_bpe * per_launch_elems}
+                "traffic": (tpe * dk["elements_per_launch"] if tpe is not None else None),
+                "algorithmic_bytes_per_launch": dk["algorithmic_bytes_per_launch"],
+                "elements_per_launch": dk["elements_per_launch"]}
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(fq, pipe, items, stream, device, args, world)
@@ -595,23 +732,32 @@ def main(argv=None):
 
     clocks = sampler.summary()
     step_ms = total_ms / args.steps
+    tags = sorted({item_tag(lbl) for lbl, *_ in items})
+    tensors = []
+    for lbl, x, *_ in items:
+        t = f"{lbl.split('/', 1)[-1]}:{x.shape[0]}x{x.shape[1]}"
+        if t not in tensors:
+            tensors.append(t)
     line = {
         "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": args.workload, "tensors": [f"{lbl}:{x.shape[0]}x{x.shape[1]}" for lbl, x, *_ in items],
-                   "format": {U4: "NVFP4 b16 UE4M3", E8: "MXFP4 b32 E8M0"}[items[0][2]] +
-                             (" + FP32 per-tensor scale" if items[0][5] == COMP else ""),
-                   "rot": items[0][4], "elements_per_step": elements_step,
+        "config": {"workload": args.workload,
+                   "tensors": tensors if len(tensors) <= 16 else
+                              f"{len(tensors)} tensors: " + ", ".join(tensors[:7]) + ", ...",
+                   "variants": tags if tags != [""] else None,
+                   "format": describe_format(items),
+                   "rot": sorted({it[4] for it in items}), "elements_per_step": elements_step,
+                   "distinct_input_bytes": distinct_bytes,
                    "block_scales": "max rule" if args.search is None else
                                    f"MSE search: max-rule code, {args.search[1]} above, {args.search[0]} below",
                    "outlier_stats": None if args.outlier_stats is None else
                                     f"max, P{100 * args.outlier_stats:g} of |x| and channel maxima per tensor",
                    "l2": "L2 flushed between steps (512 MiB write)" if in_l2 else
-                         f"inputs larger than L2 ({elements_step * 2 / 1e9:.2f} GB bf16 per step)",
+                         f"inputs larger than L2 ({distinct_bytes / 1e9:.2f} GB of distinct bf16 input)",
                    "parallelism": f"{world} independent replica(s), no data-path collective",
                    "timing": "CUDA events at step boundaries on the launching stream (value, ms_per_step); "
-                             "kernel shares from a second pass of K steps with an event after every call",
+                             f"kernel shares from {kernel_steps} more steps with an event after every call",
                    "input": "bf16 written by torch's seeded generator on the device"},
         "hbm": {"GB_per_s": step_bytes / 1e9 / (step_ms / 1e3), "bytes_per_step": step_bytes,
                 "frac_of_measured": step_bytes / 1e9 / (step_ms / 1e3) / peak,
@@ -631,24 +777,62 @@ def main(argv=None):
     return 0
 
 
+E2E_OUTPUTS = ("codes", "scales", "gscale", "bm", "terms")
+
+
 def run_e2e(fq, pipe, items, stream, device, args, world):
-    """Same step with the input in pinned host memory: H2D copy of every tensor,
-    the hot path, and a D2H read of codes, scales, G and the MSE terms."""
+    """The same step with the input in pinned host memory: every input tensor
+    copied host to device, the hot path, and every output but the dequantized
+    tensor copied back (codes, scale bytes, [amax, G], per-block MSE, tensor
+    terms).  The dequantized bf16 tensor stays in HBM, where its consumer (the
+    GEMM that the quantizer feeds) reads it.  Tensor by tensor on three streams:
+    the copy in of the next tensor and the copy out of the previous one overlap
+    the kernels of the current one."""
     import torch
-    steps = args.e2e_steps or max(3, args.steps // 20)
-    host_in = [x.cpu().pin_memory() for _, x, *_ in items]
-    host_out = [{k: torch.empty(b[k].shape, dtype=b[k].dtype, pin_memory=True)
-                 for k in ("codes", "scales", "gscale", "terms")} for b in pipe.bufs]
-    h2d = sum(h.numel() * 2 for h in host_in)
-    d2h = sum(sum(o[k].numel() * o[k].element_size() for k in o) for o in host_out)
+    steps = args.e2e_steps or WORKLOAD_DEFAULTS[args.workload]["e2e_steps"]
+    xs = {}
+    for i, (_, x, *_) in enumerate(items):
+        xs.setdefault(x.data_ptr(), (x, []))[1].append(i)
+    host_in = {}
+    for k, (x, _) in xs.items():
+        host_in[k] = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        host_in[k].copy_(x)
+    # host destinations, one set per output shape: the copy-out stream runs in order,
+    # so a set is rewritten only after its previous copy has completed
+    host_out = {}
+    for b in pipe.bufs:
+        key = tuple((k, tuple(b[k].shape), b[k].dtype) for k in E2E_OUTPUTS)
+        if key not in host_out:
+            host_out[key] = {k: torch.empty(b[k].shape, dtype=b[k].dtype, pin_memory=True) for k in E2E_OUTPUTS}
+    outs = [host_out[tuple((k, tuple(b[k].shape), b[k].dtype) for k in E2E_OUTPUTS)] for b in pipe.bufs]
+    h2d = sum(x.numel() * 2 for x, _ in xs.values())
+    d2h = sum(b[k].numel() * b[k].element_size() for b in pipe.bufs for k in E2E_OUTPUTS)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
 
     def one():
-        for (lbl, x, *_), h in zip(items, host_in):
-            x.copy_(h, non_blocking=True)
-        pipe.step(stream)
-        for b, o in zip(pipe.bufs, host_out):
-            for k in o:
-                o[k].copy_(b[k], non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(stream)
+        s_in.wait_event(start)
+        if pipe.any_comp:
+            pipe.gs_all.zero_()
+        done_out = None
+        for k, (x, idx) in xs.items():
+            with torch.cuda.stream(s_in):
+                x.copy_(host_in[k], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            stream.wait_event(ev_in)
+            pipe.run_items(idx)
+            ev_done = torch.cuda.Event()
+            ev_done.record(stream)
+            s_out.wait_event(ev_done)
+            with torch.cuda.stream(s_out):
+                for i in idx:
+                    for name in E2E_OUTPUTS:
+                        outs[i][name].copy_(pipe.bufs[i][name], non_blocking=True)
+                done_out = torch.cuda.Event()
+                done_out.record(s_out)
+        stream.wait_event(done_out)
 
     with torch.cuda.stream(stream):
         one()
@@ -661,7 +845,10 @@ def run_e2e(fq, pipe, items, stream, device, args, world):
         torch.cuda.synchronize()
     ms = reduce_max(a.elapsed_time(b), device)
     return {"value": world * pipe.elements * steps / (ms / 1e3) / 1e9, "unit": "Gelem/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "outputs_copied": list(E2E_OUTPUTS),
+            "outputs_on_device": ["the dequantized bf16 tensor (read there by its consumer)"],
+            "pipeline": "tensor by tensor: copy in, kernels and copy out on three streams"}
 
 
 if __name__ == "__main__":

@@ -51,3 +51,80 @@ def test_cpu_baseline_single_core_and_all_cores():
     ac = cb["all_cores"]
     assert "unavailable" not in ac, ac
     assert ac["value"] > 0 and 1 <= ac["cores"] <= bench.MAX_ORACLE_PROCS
+
+
+class _FakeStream:
+    cuda_stream = 0
+
+
+class _FakeLib:
+    """Stands in for libfp4q.so's entry points: records the calls a step makes."""
+
+    def __init__(self):
+        self.log = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.log.append((name, args[0]))
+            return 0
+        return fn
+
+
+class _FakeFq:
+    def __init__(self):
+        self.L = _FakeLib()
+
+    def lib(self):
+        return self.L
+
+    @staticmethod
+    def fp4q_block_mse_workspace_size(rows, cols, block):
+        return 64
+
+
+def test_weight_pass_schedule():
+    """Variant by variant, layer by layer; in each layer group the amax passes of
+    the NVFP4 variants come before the quantizer passes, and every call of
+    every item runs exactly once per step."""
+    import torch
+    xs = [(f"L{l}.{t}", torch.zeros((2, 64), dtype=torch.bfloat16)) for l in range(3) for t in "abc"]
+    items, groups = bench.weight_pass_items(xs, 3)
+    assert len(items) == 4 * 9 and len(groups) == 4 * 3
+    assert [bench.item_tag(lbl) for lbl, *_ in items[::9]] == [v[0] for v in bench.WEIGHT_PASS_VARIANTS]
+    fq = _FakeFq()
+    pipe = bench.Pipeline(fq, items, "cpu", _FakeStream(), groups=groups)
+    fq.L.log.clear()
+    pipe.step(_FakeStream())
+    names = [n for n, _ in fq.L.log]
+    n_nv = sum(1 for v in bench.WEIGHT_PASS_VARIANTS if v[4] == 1)
+    assert names.count("fp4q_tensor_amax_accumulate") == 9 * n_nv
+    assert names.count("fp4q_quantize_mse_dequantize") == 36
+    assert pipe.launches_per_step == 36 + 9 * n_nv
+    # within an NVFP4 layer group: three amax calls, then three quantizer calls on the same tensors
+    order = [(bench.stage_kind(pipe.calls[i][k][0]), i) for i, k in pipe.order]
+    nv_first = next(j for j, (kind, _) in enumerate(order) if kind == "amax")
+    grp = order[nv_first:nv_first + 6]
+    assert [k for k, _ in grp] == ["amax"] * 3 + ["quantize_mse_dequantize"] * 3
+    assert [i for _, i in grp[:3]] == [i for _, i in grp[3:]]
+    # one dequantized-output buffer per input tensor, shared by the variants
+    assert len({b["deq"].data_ptr() for b in pipe.bufs}) == 9
+    # stage names carry the variant
+    assert {bench.item_tag(lbl) for lbl, *_ in items} == {s.split("@")[1] for i, k in pipe.order
+                                                          for s in [pipe.calls[i][k][0]]}
+
+
+def test_weight_pass_and_sweep_defaults():
+    a = bench.parse_args([])
+    assert a.workload == "qwen25_14b_weight_pass" and a.steps >= 3 and a.warmup >= 3
+    a = bench.parse_args(["--workload", "block_size_sweep_4096", "--steps", "7"])
+    assert a.steps == 7 and a.warmup == bench.WORKLOAD_DEFAULTS["block_size_sweep_4096"]["warmup"]
+
+
+def test_reference_arm_sweep(capsys, monkeypatch):
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    assert bench.run_reference(bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "0",
+                                                 "--workload", "block_size_sweep_4096"])) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"]["workload"] == "block_size_sweep_4096"
