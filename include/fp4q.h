@@ -37,8 +37,8 @@
  *  - Alignment: bf16 tensors and code buffers 32 bytes; scale and per-block
  *    MSE buffers 16 bytes; gscale 4 bytes; terms and workspace 8 bytes.
  *  - Errors: invalid arguments return a negative fp4q_status before anything
- *    is enqueued.  A failed launch returns FP4Q_ERR_CUDA.  No call ever
- *    synchronizes the device.  Inputs must be finite: a block holding NaN or
+ *    is enqueued.  A failed launch returns FP4Q_ERR_CUDA.  No call but
+ *    fp4q_device_fault synchronizes the device.  Inputs must be finite: a block holding NaN or
  *    Inf gets an unspecified scale byte and codes (no fault).
  */
 #ifndef FP4Q_H
@@ -315,6 +315,57 @@ FP4Q_API int fp4q_block_mse_noalloc(const void* x, const uint8_t* codes, const u
  */
 FP4Q_API int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* stream);
 FP4Q_API int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, void* stream);
+
+/* fp4q_quantize with the scale bytes written in the layout the block-scaled
+ * tensor-core MMA reads them from (the operand layout of fp4q_gemm), for the
+ * two formats that MMA takes: MXFP4 (E8M0, block 32) and NVFP4 (UE4M3, block
+ * 16).  "Bridging the Gap", s3.4 and s4: the quantized codes and block scales
+ * feed FP4 GEMMs directly.  Codes and G are exactly fp4q_quantize's.
+ * Layout of scales_mma (fp4q_mma_scales_size bytes; rows padded to 128, the
+ * cols / block scale columns to 4): 512-byte atoms of 128 rows x 4
+ * consecutive block scales, atom (r / 128, j / 4) at byte
+ * ((r / 128) * ceil(cols / block / 4) + j / 4) * 512; inside an atom, the
+ * scale of row r (r % 128 = 32 g + i) and column j is byte i * 16 + g * 4 +
+ * j % 4.  Bytes of padding rows and columns are left as they were.  Other
+ * formats or block sizes: FP4Q_ERR_UNSUPPORTED.  Other arguments and errors
+ * as fp4q_quantize (scales_mma aligned to 16 bytes). */
+FP4Q_API int fp4q_quantize_mma(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                               uint8_t* codes, uint8_t* scales_mma, float* gscale, void* stream);
+
+/* The block-scaled FP4 GEMM that consumes two quantized operands ("Bridging
+ * the Gap", s3.4 and s4: FP4 GEMMs take the codes and block scales of both
+ * operands; "Diagnosing FP4 inference", Methodology: quantized weights feed
+ * the compute), on the tensor cores:
+ *   y[i][j] = G_A G_B sum_k q_A[i][k] s_A[i][k / b] q_B[j][k] s_B[j][k / b],
+ * q the E2M1 value of a code, s the decoded scale byte without the per-tensor
+ * scale, b = 16 (fmt UE4M3, NVFP4) or 32 (fmt E8M0, MXFP4).  A is m x k, B is
+ * n x k, both as fp4q_quantize_mma writes them: codes [rows][k / 2], scales
+ * in the MMA layout (fp4q_mma_scales_size(rows, k, b) bytes).  gscale_a /
+ * gscale_b: device pointers to G_A / G_B, or NULL for 1 (must be NULL for
+ * E8M0).  y: device fp32 [m][n], row-major, overwritten.  The products are
+ * exact and the sum is accumulated in fp32 in the tensor cores, then scaled
+ * by fp32(G_A G_B).  k % 64 == 0 (FP4Q_ERR_SHAPE otherwise); m, n >= 0 any;
+ * codes and scales 16-byte aligned, y 16-byte aligned.  k == 0 writes zeros.
+ * Enqueued on `stream`. */
+FP4Q_API int fp4q_gemm(const uint8_t* codes_a, const uint8_t* scales_a, const float* gscale_a, int64_t m,
+                       const uint8_t* codes_b, const uint8_t* scales_b, const float* gscale_b, int64_t n,
+                       int64_t k, int fmt, float* y, void* stream);
+
+/* Bytes of the block-scaled MMA scale layout for a rows x cols tensor: 512 *
+ * ceil(rows / 128) * ceil(cols / block / 4); 0 for an empty tensor. */
+FP4Q_API size_t fp4q_mma_scales_size(int64_t rows, int64_t cols, int block);
+
+/* The library's device fault word on the current device, read into
+ * *fault_out: 0 normally; 1 once a kernel that rotates on the tensor cores
+ * (rot 16 or 32 in fp4q_quantize, fp4q_quantize_mse,
+ * fp4q_quantize_mse_dequantize and fp4q_tensor_amax[_accumulate]) gave up a
+ * bounded wait for its matrix-multiply instructions instead of hanging; the
+ * outputs of that call are then incomplete.  clear != 0 resets the word to 0
+ * after reading it.  The pages have no counterpart: this is the library's own
+ * failure report.  Unlike every other entry point this call synchronizes the
+ * current device (it reads device memory).  FP4Q_ERR_NULL if fault_out is
+ * NULL; FP4Q_ERR_CUDA if the device cannot be read. */
+FP4Q_API int fp4q_device_fault(unsigned int* fault_out, int clear);
 
 /* Static text for a status code; never NULL. */
 FP4Q_API const char* fp4q_status_string(int status);

@@ -60,6 +60,10 @@ def _load() -> ctypes.CDLL:
         "fp4q_scale_encode_f32": (I, [P, I64, I, P, P]),
         "fp4q_status_string": (ctypes.c_char_p, [I]),
         "fp4q_version": (I, []),
+        "fp4q_device_fault": (I, [P, I]),
+        "fp4q_quantize_mma": (I, [P, I64, I64, I, I, I, I, P, P, P, P]),
+        "fp4q_mma_scales_size": (ctypes.c_size_t, [I64, I64, I]),
+        "fp4q_gemm": (I, [P, P, P, I64, P, P, P, I64, I64, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -117,6 +121,14 @@ def fp4q_status_string(status: int) -> str:
     return lib().fp4q_status_string(status).decode()
 
 
+def fp4q_device_fault(clear: bool = False) -> int:
+    """The library's device fault word on the current device (0, or 1 after a
+    tensor-core kernel gave up a bounded wait); synchronizes the device."""
+    out = ctypes.c_uint(0)
+    _check(lib().fp4q_device_fault(ctypes.addressof(out), int(bool(clear))), "fp4q_device_fault")
+    return int(out.value)
+
+
 def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
                   codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
                   gscale: Optional[torch.Tensor] = None, stream=None
@@ -144,6 +156,57 @@ def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
                             _ptr(gscale), _stream(stream))
     _check(st, "fp4q_quantize")
     return codes, scales, gscale
+
+
+def fp4q_mma_scales_size(rows: int, cols: int, block: int) -> int:
+    return int(lib().fp4q_mma_scales_size(rows, cols, block))
+
+
+def fp4q_quantize_mma(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
+                      codes: Optional[torch.Tensor] = None, scales_mma: Optional[torch.Tensor] = None,
+                      gscale: Optional[torch.Tensor] = None, stream=None
+                      ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """fp4q_quantize with the scale bytes in the block-scaled MMA layout (the
+    operand layout of fp4q_gemm); returns (codes, scales_mma, gscale)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    fmt, gmode = _fmt(fmt), _gmode(gmode)
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales_mma is None:
+        scales_mma = torch.zeros((max(fp4q_mma_scales_size(rows, cols, block), 1),), dtype=torch.uint8, device=dev)
+    if gscale is None and gmode == FP4Q_GLOBAL_FROM_AMAX:
+        raise ValueError("from_amax mode reads the tensor maximum from gscale[0]: pass a 2-float gscale")
+    if gscale is None and gmode != FP4Q_GLOBAL_NONE:
+        gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    _need_cuda(codes, scales_mma, gscale)
+    st = lib().fp4q_quantize_mma(_ptr(x), rows, cols, fmt, block, rot, gmode, _ptr(codes), _ptr(scales_mma),
+                                 _ptr(gscale), _stream(stream))
+    _check(st, "fp4q_quantize_mma")
+    return codes, scales_mma, gscale
+
+
+def fp4q_gemm(codes_a: torch.Tensor, scales_a: torch.Tensor, gscale_a: Optional[torch.Tensor],
+              codes_b: torch.Tensor, scales_b: torch.Tensor, gscale_b: Optional[torch.Tensor], fmt,
+              y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = G_A G_B (A . S_A)(B . S_B)^T from two fp4q_quantize_mma outputs;
+    returns y, fp32 [m][n]."""
+    m, kb = codes_a.shape
+    n, kb2 = codes_b.shape
+    if kb != kb2:
+        raise ValueError("A and B must have the same k")
+    fmt = _fmt(fmt)
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=codes_a.device)
+    _need_cuda(codes_a, scales_a, gscale_a, codes_b, scales_b, gscale_b, y)
+    st = lib().fp4q_gemm(_ptr(codes_a), _ptr(scales_a), _ptr(gscale_a), m, _ptr(codes_b), _ptr(scales_b),
+                         _ptr(gscale_b), n, 2 * kb, fmt, _ptr(y), _stream(stream))
+    _check(st, "fp4q_gemm")
+    return y
 
 
 def fp4q_quantize_search(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none", below: int = 1,

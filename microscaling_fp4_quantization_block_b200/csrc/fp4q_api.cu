@@ -179,6 +179,18 @@ extern "C" {
 
 int fp4q_version(void) { return kAbiVersion; }
 
+int fp4q_device_fault(unsigned int* fault_out, int clear)
+{
+    if (!fault_out) return FP4Q_ERR_NULL;
+    unsigned int* word = device_fault_word();
+    if (!word) return FP4Q_ERR_CUDA;
+    if (cudaMemcpy(fault_out, word, sizeof(unsigned int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    if (clear && cudaMemset(word, 0, sizeof(unsigned int)) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (clear && cudaDeviceSynchronize() != cudaSuccess) return FP4Q_ERR_CUDA;
+    return FP4Q_OK;
+}
+
 const char* fp4q_status_string(int status)
 {
     switch (status) {
@@ -197,11 +209,13 @@ const char* fp4q_status_string(int status)
 // scale search over below / above neighbouring codes.
 static int quantize_impl(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
                          uint8_t* codes, uint8_t* scales, float* gscale, bool search, int below, int above,
-                         void* stream)
+                         void* stream, bool mma_layout = false)
 {
     int64_t n = 0;
     int st = check_shape(rows, cols, fmt, block, rot, &n);
     if (st) return st;
+    if (mma_layout && !((fmt == FP4Q_SCALE_E8M0 && block == 32) || (fmt == FP4Q_SCALE_UE4M3 && block == 16)))
+        return FP4Q_ERR_UNSUPPORTED;
     if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
     if (gmode != FP4Q_GLOBAL_NONE) {
@@ -233,6 +247,10 @@ static int quantize_impl(const void* x, int64_t rows, int64_t cols, int fmt, int
     p.scales = scales;
     set_global(gmode, gscale, &p.gsrc, &p.gdst);
     rotation_constants(rot, &p.c_hi, &p.c_lo);
+    if (mma_layout) {
+        p.sf_cols = cols / block;
+        p.sf_kt = (p.sf_cols + 3) / 4;
+    }
     if (search) {
         p.below = below;
         p.above = above;
@@ -245,6 +263,20 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream)
 {
     return quantize_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, false, 0, 0, stream);
+}
+
+size_t fp4q_mma_scales_size(int64_t rows, int64_t cols, int block)
+{
+    if (rows <= 0 || cols <= 0 || block <= 0) return 0;
+    const int64_t sf_cols = cols / block;
+    return (size_t)(((rows + 127) / 128) * ((sf_cols + 3) / 4) * 512);
+}
+
+int fp4q_quantize_mma(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,
+                      uint8_t* codes, uint8_t* scales_mma, float* gscale, void* stream)
+{
+    return quantize_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales_mma, gscale, false, 0, 0, stream,
+                         true);
 }
 
 int fp4q_quantize_search(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int gmode,

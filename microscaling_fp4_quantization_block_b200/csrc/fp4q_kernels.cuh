@@ -459,7 +459,20 @@ struct QuantParams {
     float* gdst;           // G from the tensor maximum: *gsrc is that maximum, G is written here
     uint16_t* y;           // fused MSE with dequantized output: n bf16 values
     int below, above;      // scale search: codes tried below / above the max-rule code
+    unsigned int* fault;   // tensor-core kernels: set to 1 when a bounded wait gives up
+    int64_t sf_cols;       // > 0: scale bytes in the block-scaled MMA layout, sf_cols = cols / B
+    int64_t sf_kt;         //   ... with sf_kt = ceil(sf_cols / 4) 512-byte atoms per 128-row block
 };
+
+// Offset of scale byte (row r, block column j) in the block-scaled MMA layout:
+// 512-byte atoms of 128 rows x 4 consecutive block scales, atom (r / 128,
+// j / 4) at ((r / 128) sf_kt + j / 4) * 512; inside, row r % 128 = 32 g + i
+// holds its 4 bytes at i * 16 + g * 4, so each 32-bit word is one row's 4
+// scales and each 16-byte line the words of rows i, i + 32, i + 64, i + 96.
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_t sf_kt)
+{
+    return (((r >> 7) * sf_kt + (j >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (j & 3);
+}
 
 // Store a unit's code word (16 bytes; with EF evict-first in L2, for codes
 // that nothing reads again in the step) and its blocks' scale bytes; a unit
@@ -484,7 +497,19 @@ __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, cons
             for (int j = 0; j < 4; ++j)
                 if (4 * k + j < nbytes) cdst[4 * k + j] = (uint8_t)(cw[k] >> (8 * j));
     }
-    if constexpr (S::LPB > 1) {
+    if (p.sf_cols > 0) {
+        // the block-scaled MMA layout: a unit's blocks lie in one row
+        const int64_t g0 = e0 / B;
+        const int64_t r = g0 / p.sf_cols, j0 = g0 - r * p.sf_cols;
+        if constexpr (S::LPB > 1) {
+            if ((lane % S::LPB) == 0) p.scales[mma_scale_offset(r, j0, p.sf_kt)] = (uint8_t)code[0];
+        } else {
+            const int64_t nblk = p.n / B;
+#pragma unroll
+            for (int bi = 0; bi < NB; ++bi)
+                if (g0 + bi < nblk) p.scales[mma_scale_offset(r, j0 + bi, p.sf_kt)] = (uint8_t)code[bi];
+        }
+    } else if constexpr (S::LPB > 1) {
         if ((lane % S::LPB) == 0) p.scales[e0 / B] = (uint8_t)code[0];
     } else {
         const int64_t b0 = e0 / B;
@@ -506,21 +531,16 @@ __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, cons
     }
 }
 
+// Scale, codes, MSE terms, dequantized values and stores of unit u, whose
+// (rotated) values are v and whose blocks' absolute maxima are m.
 template <int FMT, int B, int K, bool MSE, bool DQ>
-__device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
-                                              int lane, const ScaleConsts& kc, const float2* tab, float nz,
-                                              double (&acc)[3], uint64_t pol)
+__device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u, const f32x2 (&v)[EPT / 2],
+                                                const float (&m)[UnitShape<B, K>::NB], int lane,
+                                                const ScaleConsts& kc, const float2* tab, float nz,
+                                                double (&acc)[3], uint64_t pol)
 {
     using S = UnitShape<B, K>;
     constexpr int NB = S::NB, BE = S::BE;
-    f32x2 v[EPT / 2];
-    unpack_unit(w, v);
-    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
-
-    float m[NB];
-    if constexpr (K == 0) block_max_words<B>(w, m);
-    else block_max<B, K>(v, m);
-
     float sc[NB], rm[NB];
     uint32_t code[NB];
     const bool exact = unit_scales<FMT, NB>(m, kc, tab, code, sc, rm);
@@ -651,6 +671,21 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
 
     // ---- stores
     store_unit<B, K, DQ>(p, u, cw, code, lane, pol);
+}
+
+template <int FMT, int B, int K, bool MSE, bool DQ>
+__device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
+                                              int lane, const ScaleConsts& kc, const float2* tab, float nz,
+                                              double (&acc)[3], uint64_t pol)
+{
+    using S = UnitShape<B, K>;
+    f32x2 v[EPT / 2];
+    unpack_unit(w, v);
+    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+    float m[S::NB];
+    if constexpr (K == 0) block_max_words<B>(w, m);
+    else block_max<B, K>(v, m);
+    quantize_values<FMT, B, K, MSE, DQ>(p, u, v, m, lane, kc, tab, nz, acc, pol);
 }
 
 // Two CTAs per SM (up to 128 registers) unless the kernel fits three without
@@ -863,6 +898,7 @@ struct AmaxParams {
     int64_t n;
     unsigned int* amax_bits;   // max |y| as fp32 bits (non-negative floats order as integers)
     float c_hi, c_lo;
+    unsigned int* fault;       // tensor-core kernel: set to 1 when a bounded wait gives up
 };
 
 template <int K>

@@ -15,6 +15,11 @@ struct MseParams;
 // and device) and return how many of its CTAs fit on the device at once.
 int resident_ctas(const void* kernel, int smem);
 
+// Device address of the library's fault word on the current device (looked up
+// once per device): the tensor-core kernels set it to 1 when a bounded wait on
+// the tensor cores gives up instead of hanging.
+unsigned int* device_fault_word();
+
 // Grid for a grid-stride kernel: min(ctas_needed, resident CTAs), at least 1.
 int grid_for(const void* kernel, int smem, int64_t ctas_needed);
 

@@ -4,8 +4,27 @@
 
 #include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
+#include "fp4q_tc.cuh"
 
 namespace fp4q {
+
+// 0 at load; a tensor-core kernel whose bounded wait on an MMA gives up sets it to 1.
+static __device__ unsigned int g_device_fault;
+
+unsigned int* device_fault_word()
+{
+    static std::mutex mu;
+    static std::unordered_map<int, unsigned int*> addr;   // device -> address of g_device_fault
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addr.find(dev);
+    if (it != addr.end()) return it->second;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_fault) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+    return static_cast<unsigned int*>(p);
+}
 
 int resident_ctas(const void* kernel, int smem)
 {
@@ -59,6 +78,18 @@ namespace {
 template <int K>
 cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
+    if constexpr (K == 16 || K == 32) {
+        // the rotation on the tensor cores: one 4096-element tile per warpgroup
+        AmaxParams q = p;
+        q.fault = device_fault_word();
+        if (q.fault == nullptr) return cudaErrorInvalidDevice;
+        auto kern = amax_tc_kernel<K>;
+        const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
+        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, (tiles + tc::WGS - 1) / tc::WGS);
+        if (pdl) return launch_pdl(kern, grid, kThreads, tc::SMEM_BYTES, s, q);
+        kern<<<grid, kThreads, tc::SMEM_BYTES, s>>>(q);
+        return cudaGetLastError();
+    }
     auto kern = amax_kernel<K>;
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));
     if (pdl) return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);

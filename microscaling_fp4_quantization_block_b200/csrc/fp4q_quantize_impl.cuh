@@ -4,6 +4,7 @@
 
 #include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
+#include "fp4q_tc.cuh"
 
 namespace fp4q {
 namespace detail {
@@ -11,6 +12,19 @@ namespace detail {
 template <int FMT, int B, int K, bool MSE, bool DQ = false>
 cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
 {
+    if constexpr (K == 16 || K == 32) {
+        // the rotation on the tensor cores: one 4096-element tile per warpgroup
+        QuantParams q = p;
+        q.fault = device_fault_word();
+        if (q.fault == nullptr) return cudaErrorInvalidDevice;
+        auto kern = quantize_tc_kernel<FMT, B, K, MSE, DQ>;
+        const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
+        int64_t need = (tiles + tc::WGS - 1) / tc::WGS;
+        if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
+        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, need);
+        if (grid_out) *grid_out = grid;
+        return launch_pdl(kern, grid, kThreads, tc::SMEM_BYTES, s, q);
+    }
     auto kern = quantize_kernel<FMT, B, K, MSE, DQ>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);

@@ -151,3 +151,33 @@ def test_binding_refuses_cpu_tensors(fp4q):
     x = torch.zeros((4, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fp4q.fp4q_quantize(x, "nvfp4", 16)
+
+
+def test_gemm_and_mma_layout_reject_bad_arguments(fp4q):
+    """fp4q_gemm and fp4q_quantize_mma reject bad arguments before any launch;
+    fp4q_mma_scales_size is 512 bytes per (128-row, 4-block) atom."""
+    L = fp4q.lib()
+    E8, U4, U5 = 0, 1, 2
+    assert L.fp4q_mma_scales_size(128, 256, 16) == 512 * 4
+    assert L.fp4q_mma_scales_size(129, 256, 16) == 512 * 4 * 2
+    assert L.fp4q_mma_scales_size(1, 64, 32) == 512          # 2 block columns pad to one atom
+    assert L.fp4q_mma_scales_size(0, 64, 32) == 0
+    g = L.fp4q_gemm
+    assert g(A32, A32, None, 128, A32, A32, None, 128, 96, E8, A32, None) == -2      # k % 64
+    assert g(A32, A32, None, -1, A32, A32, None, 128, 64, E8, A32, None) == -2
+    assert g(A32, A32, None, 128, A32, A32, None, 128, 64, U5, A32, None) == -4      # not an MMA scale type
+    assert g(A32, A32, A32, 128, A32, A32, None, 128, 64, E8, A32, None) == -4       # E8M0: no tensor scale
+    assert g(A32, A32, None, 128, A32, A32, None, 128, 64, E8, None, None) == -1
+    assert g(A32, A32, None, 128, A32, A32, None, 128, 64, E8, A32 + 4, None) == -3  # y 16-aligned
+    assert g(None, A32, None, 128, A32, A32, None, 128, 64, E8, A32, None) == -1
+    assert g(A32 + 8, A32, None, 128, A32, A32, None, 128, 64, E8, A32, None) == -3
+    assert g(A32, A32, A32 + 2, 128, A32, A32, None, 128, 64, U4, A32, None) == -3
+    assert g(None, None, None, 0, None, None, None, 128, 64, E8, None, None) == 0    # empty: nothing to do
+    qm = L.fp4q_quantize_mma
+    assert qm(A32, 4, 64, U4, 32, 0, 0, A32, A32, None, None) == -4                 # NVFP4 is block 16
+    assert qm(A32, 4, 64, E8, 16, 0, 0, A32, A32, None, None) == -4                 # MXFP4 is block 32
+    assert qm(A32, 4, 64, U5, 16, 0, 0, A32, A32, None, None) == -4
+    assert qm(A32, 4, 48, E8, 32, 0, 0, A32, A32, None, None) == -2
+    assert qm(A32, 4, 64, U4, 16, 0, 0, A32, A32 + 8, None, None) == -3
+    assert qm(None, 0, 64, U4, 16, 0, 0, None, None, None, None) == 0
+    assert L.fp4q_device_fault(None, 0) == -1

@@ -1,0 +1,85 @@
+"""The Hadamard rotation on the tensor cores (rotations of 16 and 32, "Bridging
+the Gap", s3.1: block-wise rotation fused with quantization), through the C ABI.
+
+The quantize kernels with rot 16 / 32 rotate with tcgen05.mma (bf16 operands,
+fp32 accumulators in tensor memory) instead of fp32 butterflies; the results
+obey the same rotated-path rule against the oracle's fp64 rotation.  These
+cases walk the warpgroup pipeline through its edges: one partial tile, exactly
+one and two tiles, several tiles per warpgroup (both accumulator buffers and
+both mbarrier phases reused many times), and every scale format, with the
+device fault word checked after each run.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _helpers import bf16_bits, check_rotated, gpu_run, oracle_run, assert_mse_close
+
+pytestmark = pytest.mark.gpu
+
+E8, U4, U5 = 0, 1, 2
+NONE, COMP = 0, 1
+
+
+@pytest.fixture(scope="module")
+def fq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import microscaling_fp4_quantization_block_b200 as m
+    m.lib()
+    assert m.fp4q_device_fault(clear=True) in (0, 1)
+    return m
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (3, 1024), (4, 1024), (8, 1024), (7, 4096), (300, 2048)])
+@pytest.mark.parametrize("rot", [16, 32])
+def test_tile_edges(fq, rows, cols, rot):
+    """n = 32 (one row of one partial tile), 3072, 4096 (one tile), 8192 (two),
+    28672 and 614400 elements."""
+    x, _ = workloads.student_t_outliers_bf16(rows, cols, seed=rows * cols + rot, n_outlier=min(8, cols))
+    xb = bf16_bits(x)
+    for fmt, block, gmode in [(E8, 32, NONE), (U4, 16, COMP), (U4, 8, NONE), (U5, 32, NONE)]:
+        g = gpu_run(fq, x, fmt, block, rot, gmode, want_deq=False)
+        o = oracle_run(xb, fmt, block, rot, gmode, want_mse=False, want_deq=False)
+        check_rotated(g, o, oracle.bf16_bits_to_f32(xb), fmt, block, rot)
+    assert fq.fp4q_device_fault() == 0
+
+
+@pytest.mark.parametrize("rot", [16, 32])
+def test_many_tiles_per_warpgroup_fused(fq, rot):
+    """2048 x 5120 elements: 2560 tiles, several per warpgroup; the fused
+    kernel's codes, scales, dequantized values and MSE against the oracle."""
+    x, _ = workloads.student_t_outliers_bf16(2048, 5120, seed=11 + rot)
+    xd = x.cuda()
+    xb = bf16_bits(x)
+    for fmt, block, gmode in [(E8, 32, "none"), (U4, 16, "compute")]:
+        codes, scales, gs, y, bm, terms = fq.fp4q_quantize_mse_dequantize(xd, fmt, block, rot, gmode)
+        torch.cuda.synchronize()
+        G = float(gs.item()) if gs is not None else 1.0
+        g = {"codes": codes.cpu().numpy(), "scales": scales.cpu().numpy(), "G": G}
+        o = dict(zip(("codes", "scales", "G"), oracle.quantize(xb, fmt, block, rot, COMP if gmode == "compute"
+                                                                 else NONE)))
+        check_rotated(g, o, oracle.bf16_bits_to_f32(xb), fmt, block, rot)
+        # the dequantized output is the dequantization of the GPU's own codes
+        want = oracle.dequantize(g["codes"], g["scales"], G, 2048, 5120, fmt, block, 0)
+        got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got, oracle.f32_to_bf16_bits(want))
+        o_bm, o_terms = oracle.block_mse(xb, g["codes"], g["scales"], G, fmt, block, rot)
+        assert_mse_close(bm.cpu().numpy(), terms.cpu().numpy(), o_bm, o_terms, 1e-5)
+    assert fq.fp4q_device_fault() == 0
+
+
+@pytest.mark.parametrize("rot", [16, 32])
+def test_rotated_amax(fq, rot):
+    """max |y| over the tensor-core rotation against the exact rotation: equal up
+    to the rotation's rounding."""
+    x, _ = workloads.student_t_outliers_bf16(1000, 2048, seed=rot)
+    amax = fq.fp4q_tensor_amax(x.cuda(), rot)
+    torch.cuda.synchronize()
+    xf = oracle.bf16_bits_to_f32(bf16_bits(x))
+    want = oracle.tensor_amax(oracle.hadamard(xf, rot))
+    l1 = np.abs(xf.astype(np.float64)).reshape(-1, rot).sum(1).max() / np.sqrt(rot)
+    assert abs(float(amax.item()) - want) <= (np.log2(rot) + 2) * 2.0 ** -24 * l1 + 2.0 ** -23 * want
+    assert fq.fp4q_device_fault() == 0
