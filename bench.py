@@ -50,7 +50,11 @@ WORKLOAD_DEFAULTS = {
     "rotated_activations_8192x5120": dict(steps=200, warmup=10, e2e_steps=10),
     "block_size_sweep_4096": dict(steps=100, warmup=5, e2e_steps=5),
     "mxfp4_gaussian_1024x1024": dict(steps=200, warmup=10, e2e_steps=10),
+    "fp4_gemm_8192x13824x5120": dict(steps=50, warmup=5, e2e_steps=3),
 }
+# Nominal dense FP4 / bf16 tensor throughput of B200 (9 / 2.25 PFLOP/s): the
+# factor that turns the measured bf16 GEMM peak into the FP4 GEMM's peak.
+FP4_PER_BF16 = 4.0
 # The four variants of the whole-model weight pass: (name, fmt, block, rot, gmode).
 WEIGHT_PASS_VARIANTS = (("mxfp4_rot0", 0, 32, 0, 0), ("nvfp4_rot0", 1, 16, 0, 1),
                         ("mxfp4_rot32", 0, 32, 32, 0), ("nvfp4_rot32", 1, 16, 32, 1))
@@ -415,6 +419,16 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def measured_bf16_tflops():
+    """The measured bf16 GEMM peak (burst: a kernel timed alone), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def csrc_hash(files=None) -> str:
     """Hash of the named kernel sources (all of csrc/ when files is None)."""
     h = hashlib.sha256()
@@ -623,8 +637,153 @@ def describe_format(items):
     return seen if len(seen) > 1 else seen[0]
 
 
+GEMM_SHAPE = (8192, 13824, 5120)       # tokens x out-features x in-features (Qwen2.5-14B gate/up projection)
+
+
+def gemm_operands(device, rank, fmt_name):
+    """Activations [8192, 5120] (Student-t, outlier channels) and weights
+    [13824, 5120] (N(0, 0.02^2)), bf16 on `device`."""
+    import workloads as W
+    m, n, k = GEMM_SHAPE
+    a, _ = W.student_t_outliers_bf16(m, k, rank_seed(91, rank), device=device)
+    b = W.gaussian_bf16(n, k, 0.02, rank_seed(92, rank), device)
+    return a, b
+
+
+def run_gemm_reference(args):
+    """The oracle's FP4 GEMM on a bounded sample: the first rows of both operands."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads as W
+    m, n, k = 16, 64, GEMM_SHAPE[2]
+    fmt, block = (U4, 16) if args.fmt == "nvfp4" else (E8, 32)
+    a, _ = W.student_t_outliers_bf16(m, k, 91)
+    b = W.gaussian_bf16(n, k, 0.02, 92)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    gm = COMP if fmt == U4 else NONE
+    ca, sa, ga = oracle.quantize(bits(a), fmt, block, 0, gm)
+    cb, sb, gb = oracle.quantize(bits(b), fmt, block, 0, gm)
+    for _ in range(args.warmup):
+        oracle.fp4_gemm(ca, sa, ga, cb, sb, gb, k, fmt, block)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fp4_gemm(ca, sa, ga, cb, sb, gb, k, fmt, block)
+    dt = time.perf_counter() - t0
+    return 2.0 * m * n * k * args.steps / dt / 1e12, f"{m} x {n} x {k} per step, single-threaded C, fp64"
+
+
+def run_gemm(args):
+    """The block-scaled FP4 GEMM consumer on quantized operands: TFLOP/s."""
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        v, sample = run_gemm_reference(args)
+        print(json.dumps({"metric": "TFLOP/s of the block-scaled FP4 GEMM consumer", "value": v,
+                          "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "impl": "reference", "config": {"workload": args.workload},
+                          "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+    import torch
+
+    import microscaling_fp4_quantization_block_b200 as fq
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl", device)
+    import torch.distributed as dist
+    m, n, k = GEMM_SHAPE
+    fmt, block = (U4, 16) if args.fmt == "nvfp4" else (E8, 32)
+    gm = "compute" if fmt == U4 else "none"
+    a, b = gemm_operands(device, rank, args.fmt)
+    ca, sa, ga = fq.fp4q_quantize_mma(a, fmt, block, 0, gm)
+    cb, sb, gb = fq.fp4q_quantize_mma(b, fmt, block, 0, gm)
+    y = torch.empty((m, n), dtype=torch.float32, device=device)
+    del a, b
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())
+    L = fq.lib()
+    call = (ca.data_ptr(), sa.data_ptr(), None if ga is None else ga.data_ptr(), m, cb.data_ptr(), sb.data_ptr(),
+            None if gb is None else gb.data_ptr(), n, k, fmt, y.data_ptr(), stream.cuda_stream)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            assert L.fp4q_gemm(*call) == 0
+            flush.zero_()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler, torch.cuda.stream(stream):
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            L.fp4q_gemm(*call)
+            ev[i][1].record(stream)
+            flush.zero_()            # operands (60 MB) fit in L2: flushed between steps
+        torch.cuda.synchronize()
+    ms = reduce_max(sum(x.elapsed_time(z) for x, z in ev), device)
+    flops = 2.0 * m * n * k
+    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    per = ms / args.steps
+    bf16, kind = measured_bf16_tflops()
+    peak = FP4_PER_BF16 * bf16
+    # end to end: operands copied in from pinned host memory, y copied back
+    hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t) for t in (ca, sa, cb, sb)]
+    hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    e2e_steps = args.e2e_steps or WORKLOAD_DEFAULTS[args.workload]["e2e_steps"]
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for h, d in zip(hin, (ca, sa, cb, sb)):
+                d.copy_(h, non_blocking=True)
+            L.fp4q_gemm(*call)
+            hy.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample = run_gemm_reference(argparse.Namespace(fmt=args.fmt, warmup=1, steps=3))
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample}
+    line = {
+        "metric": "TFLOP/s of the block-scaled FP4 GEMM consumer", "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": args.workload, "m": m, "n": n, "k": k,
+                   "format": "NVFP4 b16 UE4M3 + FP32 per-tensor scale" if fmt == U4 else "MXFP4 b32 E8M0",
+                   "operands": "A: Student-t activations with outlier channels, B: N(0, 0.02^2) weights, "
+                               "quantized by fp4q_quantize_mma (untimed)",
+                   "l2": "L2 flushed between steps (512 MiB write)", "tile": "128 x 128 x 256, 1 CTA per tile"},
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel", "achieved": value / world, "peak": peak,
+                     "peak_kind": f"{kind} bf16 x {FP4_PER_BF16:g} (nominal FP4 / bf16 dense ratio)",
+                     "unit": "TFLOP/s", "frac": value / world / peak, "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+                "d2h_bytes_per_step": hy.numel() * 4, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload.startswith("fp4_gemm"):
+        return run_gemm(args)
     if args.impl == "reference":
         return run_reference(args)
     import torch

@@ -261,39 +261,10 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_gemm_kernel(const __grid_const
     }
 }
 
-// cuTensorMapEncodeTiled from the driver, fetched once (the library links the
-// runtime only).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
 bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k)
 {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)BM};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_tensor_map_2d(map, 1, codes, (uint64_t)(k / 2), (uint64_t)rows, (uint64_t)(k / 2), BKB, BM,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace gemm

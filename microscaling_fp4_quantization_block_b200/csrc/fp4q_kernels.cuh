@@ -245,9 +245,11 @@ __device__ __forceinline__ float group_sum(float s)
 
 // Per-CTA reduction of four fp64 accumulators into partials[blockIdx.x][4], in a
 // fixed order (warp butterflies, then warps in index order): deterministic.
+template <int NT = kThreads>
 __device__ __forceinline__ void cta_partials(double a0, double a1, double a2, double a3, double* partials)
 {
-    __shared__ double red[kWarps][4];
+    constexpr int NW = NT / 32;
+    __shared__ double red[NW][4];
 #pragma unroll
     for (int d = 16; d >= 1; d >>= 1) {
         a0 += __shfl_xor_sync(0xffffffffu, a0, d);
@@ -265,7 +267,7 @@ __device__ __forceinline__ void cta_partials(double a0, double a1, double a2, do
     __syncthreads();
     if (threadIdx.x < 4) {
         double s = 0.0;
-        for (int k = 0; k < kWarps; ++k) s += red[k][threadIdx.x];
+        for (int k = 0; k < NW; ++k) s += red[k][threadIdx.x];
         partials[(int64_t)blockIdx.x * 4 + threadIdx.x] = s;
     }
 }
@@ -276,8 +278,10 @@ __device__ __forceinline__ void cta_partials(double a0, double a1, double a2, do
 // order (deterministic), writes terms[i] = sum / n, and atomicInc's wrap-around
 // leaves the counter at 0 for the next call.  The counter must be 0 when the
 // kernel starts.
+template <int NT = kThreads>
 __device__ __forceinline__ void finish_partials(const double* partials, unsigned int* done, int64_t n, double* terms)
 {
+    constexpr int NW = NT / 32;
     __shared__ bool last;
     __threadfence();
     __syncthreads();
@@ -285,9 +289,9 @@ __device__ __forceinline__ void finish_partials(const double* partials, unsigned
     __syncthreads();
     if (!last) return;
     __threadfence();
-    __shared__ double red[kWarps][4];
+    __shared__ double red[NW][4];
     double s[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += kThreads)
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT)
 #pragma unroll
         for (int k = 0; k < 4; ++k) s[k] += __ldcg(partials + (int64_t)i * 4 + k);
 #pragma unroll
@@ -301,7 +305,7 @@ __device__ __forceinline__ void finish_partials(const double* partials, unsigned
     __syncthreads();
     if (threadIdx.x < 4) {
         double t = 0.0;
-        for (int w = 0; w < kWarps; ++w) t += red[w][threadIdx.x];
+        for (int w = 0; w < NW; ++w) t += red[w][threadIdx.x];
         terms[threadIdx.x] = t / (double)n;
     }
 }

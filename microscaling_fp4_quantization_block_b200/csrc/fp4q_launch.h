@@ -13,15 +13,24 @@ struct MseParams;
 
 // Opt a kernel in to `smem` bytes of dynamic shared memory (once per kernel
 // and device) and return how many of its CTAs fit on the device at once.
-int resident_ctas(const void* kernel, int smem);
+int resident_ctas(const void* kernel, int smem, int threads = 256);
 
 // Device address of the library's fault word on the current device (looked up
 // once per device): the tensor-core kernels set it to 1 when a bounded wait on
 // the tensor cores gives up instead of hanging.
 unsigned int* device_fault_word();
 
+// A 2-D TMA tensor map (driver's cuTensorMapEncodeTiled, fetched once at run
+// time): inner dimension `inner` elements of `elem_bytes` bytes, `rows` rows
+// `row_bytes` apart, boxes of box_inner x box_rows, the given swizzle
+// (CUtensorMapSwizzle value), zero fill out of bounds.  `map` points to a
+// 64-byte aligned 128-byte CUtensorMap.  False if the encoder is unavailable
+// or rejects the arguments.
+bool encode_tensor_map_2d(void* map, int elem_bytes, const void* base, uint64_t inner, uint64_t rows,
+                          uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle);
+
 // Grid for a grid-stride kernel: min(ctas_needed, resident CTAs), at least 1.
-int grid_for(const void* kernel, int smem, int64_t ctas_needed);
+int grid_for(const void* kernel, int smem, int64_t ctas_needed, int threads = 256);
 
 // CTAs a ring kernel needs for n elements (one 32-unit tile per warp).
 int64_t ring_ctas_needed(int64_t n, int ept);

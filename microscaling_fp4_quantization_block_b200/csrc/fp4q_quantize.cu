@@ -1,4 +1,5 @@
 // fp4q_quantize.cu -- launch helpers, format dispatch of quantize, and the amax kernels.
+#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
@@ -26,13 +27,49 @@ unsigned int* device_fault_word()
     return static_cast<unsigned int*>(p);
 }
 
-int resident_ctas(const void* kernel, int smem)
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+}  // namespace
+
+bool encode_tensor_map_2d(void* map, int elem_bytes, const void* base, uint64_t inner, uint64_t rows,
+                          uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || rows == 0 || inner == 0) return false;
+    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(static_cast<CUtensorMap*>(map), dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, static_cast<CUtensorMapSwizzle>(swizzle),
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int resident_ctas(const void* kernel, int smem, int threads)
 {
     static std::mutex mu;
     static std::unordered_map<uint64_t, int> cache;   // (kernel, device) -> resident CTAs
     int dev = 0;
     cudaGetDevice(&dev);
-    const uint64_t key = reinterpret_cast<uint64_t>(kernel) * 64u + (uint64_t)dev;
+    const uint64_t key = (reinterpret_cast<uint64_t>(kernel) * 64u + (uint64_t)dev) * 4096u + (uint64_t)threads;
     {
         std::lock_guard<std::mutex> lock(mu);
         auto it = cache.find(key);
@@ -41,16 +78,16 @@ int resident_ctas(const void* kernel, int smem)
     if (smem > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     int sms = 0, occ = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem);
     const int resident = (sms > 0 ? sms : 1) * (occ > 0 ? occ : 1);
     std::lock_guard<std::mutex> lock(mu);
     cache[key] = resident;
     return resident;
 }
 
-int grid_for(const void* kernel, int smem, int64_t ctas_needed)
+int grid_for(const void* kernel, int smem, int64_t ctas_needed, int threads)
 {
-    const int resident = resident_ctas(kernel, smem);
+    const int resident = resident_ctas(kernel, smem, threads);
     if (ctas_needed < 1) ctas_needed = 1;
     return (int)(ctas_needed < resident ? ctas_needed : resident);
 }
@@ -79,15 +116,20 @@ template <int K>
 cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
     if constexpr (K == 16 || K == 32) {
-        // the rotation on the tensor cores: one 4096-element tile per warpgroup
-        AmaxParams q = p;
-        q.fault = device_fault_word();
-        if (q.fault == nullptr) return cudaErrorInvalidDevice;
+        // the rotation on the tensor cores: 4096-element tiles through a TMA ring
+        TcAmaxParams tp;
+        memset(&tp, 0, sizeof(tp));
+        tp.p = p;
+        tp.p.fault = device_fault_word();
+        if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
+        if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
+                                  tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
         auto kern = amax_tc_kernel<K>;
         const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
-        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, (tiles + tc::WGS - 1) / tc::WGS);
-        if (pdl) return launch_pdl(kern, grid, kThreads, tc::SMEM_BYTES, s, q);
-        kern<<<grid, kThreads, tc::SMEM_BYTES, s>>>(q);
+        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, tiles, tc::THREADS);
+        if (pdl) return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
+        kern<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(tp);
         return cudaGetLastError();
     }
     auto kern = amax_kernel<K>;

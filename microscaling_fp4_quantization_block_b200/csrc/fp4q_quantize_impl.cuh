@@ -2,6 +2,8 @@
 // scale format (each format is its own translation unit, built in parallel).
 #pragma once
 
+#include <cstring>
+
 #include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
 #include "fp4q_tc.cuh"
@@ -13,17 +15,21 @@ template <int FMT, int B, int K, bool MSE, bool DQ = false>
 cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
 {
     if constexpr (K == 16 || K == 32) {
-        // the rotation on the tensor cores: one 4096-element tile per warpgroup
-        QuantParams q = p;
-        q.fault = device_fault_word();
-        if (q.fault == nullptr) return cudaErrorInvalidDevice;
+        // the rotation on the tensor cores: 4096-element tiles through a TMA ring
+        TcQuantParams tp;
+        memset(&tp, 0, sizeof(tp));
+        tp.p = p;
+        tp.p.fault = device_fault_word();
+        if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
+        if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
+                                  tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
         auto kern = quantize_tc_kernel<FMT, B, K, MSE, DQ>;
-        const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
-        int64_t need = (tiles + tc::WGS - 1) / tc::WGS;
+        int64_t need = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
         if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
-        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, need);
+        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, need, tc::THREADS);
         if (grid_out) *grid_out = grid;
-        return launch_pdl(kern, grid, kThreads, tc::SMEM_BYTES, s, q);
+        return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
     }
     auto kern = quantize_kernel<FMT, B, K, MSE, DQ>;
     int64_t need = ring_ctas_needed(p.n, EPT);

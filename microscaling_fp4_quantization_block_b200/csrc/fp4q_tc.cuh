@@ -13,19 +13,26 @@
 // with fp32 accumulators in tensor memory (TMEM).  Every product is exact (a
 // bf16 value times +-1) and only the accumulation rounds; the result is then
 // scaled by 1/sqrt(K) exactly as the butterfly path scales it.  Row m of D
-// lands in TMEM lane m, so after one tcgen05.ld each thread of a warpgroup
+// lands in TMEM lane m, so after one tcgen05.ld each thread of a consumer warp
 // holds the 32 rotated values of "its" row: the same 32-element unit the
 // quantizer works on, with no shuffles.
 //
-// Pipeline (per warpgroup of 128 threads, independent of the other warpgroup
-// of the CTA): a ring of NSTAGE tiles in shared memory filled by 16-byte
-// cp.async copies straight into the 64-byte-swizzled K-major layout the MMA
-// reads; one thread issues the two K=16 MMAs of tile i+1 into one of two TMEM
-// buffers while all threads read and quantize tile i from the other.  MMA
-// completion is tracked by tcgen05.commit on an mbarrier; every wait on it is
-// bounded and, when the bound runs out, records a fault (fp4q_device_fault)
-// and stops the warpgroup's work without hanging.
+// Warp-specialised pipeline (a CTA of 4 consumer warps and 1 control warp):
+//   control warp, lane 0: TMA loads of 4096-element tiles (a 2-D tensor map
+//     of 64-byte rows with the 64-byte swizzle, which is the K-major layout
+//     the MMA reads) into a ring of NSTAGE shared-memory stages, completing on
+//     the stage's `full` mbarrier;
+//   control warp, lane 1: per tile, the two K = 16 MMAs into one of NBUF TMEM
+//     accumulator buffers, then tcgen05.commit on the stage's `empty` barrier
+//     (the stage may be refilled) and the buffer's `tfull` barrier;
+//   consumer warps: per tile, wait for `tfull`, tcgen05.ld their 32 lanes,
+//     arrive on the buffer's `tempty` barrier (4 arrivals free it), quantize.
+// No barrier couples the consumer warps to one another, so each runs ahead as
+// far as the pipeline allows.  Every wait is bounded; one that runs out sets
+// the library's fault word (fp4q_device_fault) and that role stops its work.
 #pragma once
+
+#include <cuda.h>
 
 #include "fp4q_kernels.cuh"
 
@@ -33,17 +40,18 @@ namespace fp4q {
 namespace tc {
 
 constexpr int KR = 32;                          // elements per MMA row
-constexpr int ROWS = 128;                       // rows per tile (M of the MMA), one per thread of a warpgroup
+constexpr int ROWS = 128;                       // rows per tile (M of the MMA), one per consumer thread
 constexpr int TILE_ELEMS = ROWS * KR;           // 4096
 constexpr int STAGE_BYTES = ROWS * KR * 2;      // 8 KiB of bf16
-constexpr int NSTAGE = 4;                       // ring stages per warpgroup
-constexpr int WGS = kThreads / 128;             // warpgroups per CTA (2)
-constexpr int TMEM_COLS_WG = 2 * KR;            // two fp32 accumulator buffers of 32 columns
-constexpr int TMEM_COLS = WGS * TMEM_COLS_WG;   // 128 (a power of two >= 32)
+constexpr int NSTAGE = 6;                       // shared-memory ring stages
+constexpr int NBUF = 4;                         // TMEM accumulator buffers of 32 columns
+constexpr int CONSUMER_WARPS = 4;
+constexpr int THREADS = 32 * (CONSUMER_WARPS + 1);
+constexpr int TMEM_COLS = NBUF * KR;            // 128 (a power of two >= 32)
 constexpr int B_BYTES = KR * KR * 2;            // the rotation matrix, 2 KiB
 // dynamic shared memory: 1 KiB of slack to align the swizzled buffers to 1 KiB,
-// the rotation matrix, the rings, then mbarriers and the TMEM address slot
-constexpr int SMEM_BYTES = 1024 + B_BYTES + WGS * NSTAGE * STAGE_BYTES + 64;
+// the rotation matrix, the ring, then the mbarriers and the TMEM address slot
+constexpr int SMEM_BYTES = 1024 + B_BYTES + NSTAGE * STAGE_BYTES + 8 * (2 * NSTAGE + 2 * NBUF) + 16;
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
 // A and B bf16 (bits 7-9, 10-12 = 1), both K-major (bits 15, 16 = 0),
@@ -172,163 +180,154 @@ __device__ __forceinline__ void fill_rotation_matrix(uint32_t b_smem)
 }
 
 // ---------------------------------------------------------------- the pipeline
-// Every tile of 4096 elements of x (bf16, n elements, n a multiple of 32) is
-// rotated by the tensor cores; body(u, v) is then called by every thread for
-// unit u (32 consecutive elements, index u = tile * 128 + row) with the
-// rotated, not yet normalised, values v.  Rows at or past n hold zeros.
-// Warpgroups walk tiles in a grid-stride loop (the same trip count for every
-// thread of a warpgroup).  Returns false when an MMA wait gave up.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+// Bounded wait on an mbarrier phase; false (and the fault word set) when it runs out.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsigned int* fault)
+{
+    for (uint32_t polls = 0; polls < kMaxPolls; ++polls)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicExch(fault, 1u);
+    return false;
+}
+
+// Every 4096-element tile of x (bf16, n elements, n a multiple of 32, read
+// through the tensor map xmap: rows of 32 elements, boxes of 128 rows) is
+// rotated by the tensor cores; body(u, v) is then called by every consumer
+// thread for unit u (32 consecutive elements, u = tile * 128 + row) with the
+// rotated, not yet normalised, values v.  Rows at or past n read as zeros.
+// CTAs walk tiles in a grid-stride loop.  Called by all THREADS threads.
 template <int K, typename Body>
-__device__ __forceinline__ bool rotate_tiles(const uint16_t* __restrict__ x, int64_t n, uint8_t* smem_raw,
-                                             unsigned int* fault, Body&& body, bool ef, uint64_t pol)
+__device__ __forceinline__ void rotate_tiles(const void* xmap, int64_t n, uint8_t* smem_raw, unsigned int* fault,
+                                             Body&& body)
 {
     const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;               // swizzle atoms need 1 KiB alignment
     const uint32_t b_smem = base;
-    const int wg = threadIdx.x >> 7;
-    const int t128 = threadIdx.x & 127;
-    const int warp_in_wg = t128 >> 5, lane = threadIdx.x & 31;
-    const uint32_t ring = base + B_BYTES + (uint32_t)(wg * NSTAGE * STAGE_BYTES);
-    const uint32_t bars = base + B_BYTES + (uint32_t)(WGS * NSTAGE * STAGE_BYTES);     // 2 per warpgroup
-    const uint32_t bar0 = bars + 16u * (uint32_t)wg;
-    const uint32_t slot = bars + 16u * WGS;                                         // TMEM base address
-    __shared__ int abort_flag[WGS];
+    const uint32_t ring = base + B_BYTES;
+    const uint32_t bars = ring + NSTAGE * STAGE_BYTES;
+    const uint32_t full0 = bars, empty0 = full0 + 8u * NSTAGE;
+    const uint32_t tfull0 = empty0 + 8u * NSTAGE, tempty0 = tfull0 + 8u * NBUF;
+    const uint32_t slot = tempty0 + 8u * NBUF;                  // TMEM base address
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     fill_rotation_matrix<K>(b_smem);
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2 * WGS; ++i) mbar_init(bars + 8u * (uint32_t)i, 1u);
+        for (int i = 0; i < NSTAGE; ++i) {
+            mbar_init(full0 + 8u * i, 1u);
+            mbar_init(empty0 + 8u * i, 1u);
+        }
+        for (int i = 0; i < NBUF; ++i) {
+            mbar_init(tfull0 + 8u * i, 1u);
+            mbar_init(tempty0 + 8u * i, (uint32_t)CONSUMER_WARPS);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (t128 == 0) abort_flag[wg] = 0;
-    if (threadIdx.x < 32) tmem_alloc(slot, TMEM_COLS);
+    if (warp == CONSUMER_WARPS) tmem_alloc(slot, TMEM_COLS);
     fence_proxy_async_smem();                                    // the rotation matrix, for the MMA
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     uint32_t tmem_base;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem_base) : "r"(slot) : "memory");
-    const uint32_t tmem_wg = tmem_base + (uint32_t)(wg * TMEM_COLS_WG);
-    const uint32_t tmem_lane = (uint32_t)(32 * warp_in_wg) << 16;
-
-    // this thread's 4 copies of a tile: chunk g = 32 c + lane of its warp's 2 KiB
-    uint32_t s_off[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int g = 32 * c + lane;
-        s_off[c] = sw64_offset(32 * warp_in_wg + (g >> 2), g & 3);
-    }
-    const int64_t nbytes = 2 * n;
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(x);
-    auto issue = [&](int64_t tile, int stage) {
-        const uint32_t sb = ring + (uint32_t)(stage * STAGE_BYTES);
-        const int64_t off0 = tile * (int64_t)STAGE_BYTES + 2048 * warp_in_wg + 16 * lane;
-        if (off0 - 16 * lane + 2048 <= nbytes) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (ef) cp_async16(sb + s_off[c], src + off0 + 512 * c, 16u, pol);
-                else cp_async16(sb + s_off[c], src + off0 + 512 * c, 16u);
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int64_t o = off0 + 512 * c;
-                const int64_t left = nbytes - o;
-                const uint32_t cnt = left >= 16 ? 16u : (left > 0 ? (uint32_t)left : 0u);
-                cp_async16(sb + s_off[c], cnt ? (const void*)(src + o) : (const void*)src, cnt);
-            }
-        }
-    };
 
     const int64_t n_tiles = (n + TILE_ELEMS - 1) / TILE_ELEMS;
-    const int64_t first = (int64_t)blockIdx.x * WGS + wg;
-    const int64_t stride = (int64_t)gridDim.x * WGS;
-    const bool leader = t128 == 0;
-    bool ok = true;
+    const int64_t first = blockIdx.x, stride = gridDim.x;
 
-    auto issue_mma = [&](int stage, int buf) {
-        const uint32_t a = ring + (uint32_t)(stage * STAGE_BYTES);
-        const uint32_t d = tmem_wg + (uint32_t)(buf * KR);
-        tc_fence_after();
-        mma_bf16(d, sw64_desc(a), sw64_desc(b_smem), kIdescBf16F32, false);
-        mma_bf16(d, sw64_desc(a + 32u), sw64_desc(b_smem + 32u), kIdescBf16F32, true);
-        mma_commit(bar0 + 8u * (uint32_t)buf);
-    };
-
-    // prologue: NSTAGE - 1 tiles in flight, then the MMA of the first one
-#pragma unroll
-    for (int s = 0; s < NSTAGE - 1; ++s) {
-        const int64_t t = first + s * stride;
-        if (t < n_tiles) issue(t, s);
-        cp_async_commit();
-    }
-    if (first < n_tiles) {
-        cp_async_wait<NSTAGE - 2>();
-        fence_proxy_async_smem();
-        wg_sync(wg);
-        if (leader) issue_mma(0, 0);
-    }
-    int64_t i = 0;
-    for (int64_t t = first; t < n_tiles; t += stride, ++i) {
-        // refill the stage tile i - 1 used (its MMA has completed: waited below)
-        const int64_t t_fill = t + (NSTAGE - 1) * stride;
-        if (t_fill < n_tiles) issue(t_fill, (int)((i + NSTAGE - 1) % NSTAGE));
-        cp_async_commit();
-        // the MMA of tile i + 1, once every thread's copies of it have landed and
-        // every thread has read TMEM buffer (i + 1) % 2 (tile i - 1)
-        cp_async_wait<NSTAGE - 2>();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        wg_sync(wg);
-        const bool go = ok && abort_flag[wg] == 0;         // one shared load per warp: warp-uniform
-        if (leader && go && t + stride < n_tiles) issue_mma((int)((i + 1) % NSTAGE), (int)((i + 1) & 1));
-        // tile i: wait (bounded) for its MMA, then read this thread's row; the
-        // decision is made per warp, since tcgen05.ld needs the whole warp
-        bool have = false;
-        if (go) {
-            const uint32_t bar = bar0 + 8u * (uint32_t)(i & 1);
-            const uint32_t parity = (uint32_t)((i >> 1) & 1);
-            bool done = mbar_try_wait(bar, parity);
-            for (uint32_t polls = 1; !done && polls < kMaxPolls; ++polls) done = mbar_try_wait(bar, parity);
-            have = __all_sync(0xffffffffu, done);
-            if (!have) {
-                ok = false;
-                if (lane == 0) {
-                    atomicExch(fault, 1u);
-                    abort_flag[wg] = 1;
-                }
+    if (warp == CONSUMER_WARPS) {
+        if (lane == 0) {
+            // ---- TMA producer
+            int64_t i = 0;
+            for (int64_t t = first; t < n_tiles; t += stride, ++i) {
+                const int s = (int)(i % NSTAGE);
+                if (i >= NSTAGE && !wait_bounded(empty0 + 8u * s, (uint32_t)(((i / NSTAGE) - 1) & 1), fault)) break;
+                mbar_expect_tx(full0 + 8u * s, (uint32_t)STAGE_BYTES);
+                tma_load_2d(ring + (uint32_t)(s * STAGE_BYTES), xmap, 0, (int)(t * ROWS), full0 + 8u * s);
+            }
+        } else if (lane == 1) {
+            // ---- MMA issuer
+            int64_t i = 0;
+            for (int64_t t = first; t < n_tiles; t += stride, ++i) {
+                const int s = (int)(i % NSTAGE), b = (int)(i % NBUF);
+                if (!wait_bounded(full0 + 8u * s, (uint32_t)((i / NSTAGE) & 1), fault)) break;
+                if (i >= NBUF && !wait_bounded(tempty0 + 8u * b, (uint32_t)(((i / NBUF) - 1) & 1), fault)) break;
+                tc_fence_after();
+                const uint32_t a = ring + (uint32_t)(s * STAGE_BYTES);
+                const uint32_t d = tmem_base + (uint32_t)(b * KR);
+                mma_bf16(d, sw64_desc(a), sw64_desc(b_smem), kIdescBf16F32, false);
+                mma_bf16(d, sw64_desc(a + 32u), sw64_desc(b_smem + 32u), kIdescBf16F32, true);
+                mma_commit(empty0 + 8u * s);                    // the stage may be refilled
+                mma_commit(tfull0 + 8u * b);                    // the buffer may be read
             }
         }
-        if (have) {
+        __syncwarp();
+    } else {
+        // ---- consumers: warp w reads TMEM lanes 32 w .. 32 w + 31 (rows of the tile)
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        int64_t i = 0;
+        for (int64_t t = first; t < n_tiles; t += stride, ++i) {
+            const int b = (int)(i % NBUF);
+            const bool done = mbar_try_wait(tfull0 + 8u * b, (uint32_t)((i / NBUF) & 1)) ||
+                              wait_bounded(tfull0 + 8u * b, (uint32_t)((i / NBUF) & 1), fault);
+            if (!__all_sync(0xffffffffu, done)) break;         // warp-uniform: tcgen05.ld needs the warp
             tc_fence_after();
             uint32_t r[32];
-            tmem_ld32(tmem_wg + tmem_lane + (uint32_t)((i & 1) * KR), r);
+            tmem_ld32(tmem_base + lane_off + (uint32_t)(b * KR), r);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty0 + 8u * b);      // this warp is done with the buffer
             f32x2 v[EPT / 2];
 #pragma unroll
             for (int k = 0; k < EPT / 2; ++k) v[k] = pk(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
-            body(t * ROWS + t128, v);
+            body(t * ROWS + 32 * warp + lane, v);
         }
     }
-    cp_async_wait_all();
-    // every MMA this warpgroup issued has completed (each was waited on, or the
-    // warpgroup gave up), so TMEM can be released
+    // every MMA issued has completed (each was waited on by the consumers, or a
+    // role gave up), so TMEM can be released
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x < 32) {
+    if (warp == CONSUMER_WARPS) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
-    return ok;
 }
 
 }  // namespace tc
 
 // ---------------------------------------------------------------- kernels on the tensor-core rotation
+// Parameters: the quantizer's (or the maximum's) plus the tensor map of x.
+struct TcQuantParams {
+    CUtensorMap xmap;
+    QuantParams p;
+};
+
+struct TcAmaxParams {
+    CUtensorMap xmap;
+    AmaxParams p;
+};
+
 // Quantize (+ fused MSE / dequantized output) with the rotation (K = 16, 32)
 // on the tensor cores; outputs identical in layout to quantize_kernel's.
 template <int FMT, int B, int K, bool MSE, bool DQ>
-__global__ void __launch_bounds__(kThreads, 2) quantize_tc_kernel(QuantParams p)
+__global__ void __launch_bounds__(tc::THREADS, 3) quantize_tc_kernel(const __grid_constant__ TcQuantParams tp)
 {
     static_assert(K == 16 || K == 32, "tensor-core rotation of 16 or 32");
+    const QuantParams& p = tp.p;
     pdl_wait();
     pdl_release();
     extern __shared__ __align__(128) uint8_t smem_tc[];
@@ -349,18 +348,15 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_tc_kernel(QuantParams p)
     const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
     double acc[3] = {0.0, 0.0, 0.0};
     const uint64_t pol = l2_evict_first();
-    tc::rotate_tiles<K>(
-        p.x, p.n, smem_tc, p.fault,
-        [&](int64_t u, f32x2 (&v)[EPT / 2]) {
-            normalize<EPT>(v, p.c_hi, p.c_lo);
-            float m[UnitShape<B, K>::NB];
-            block_max<B, K>(v, m);
-            quantize_values<FMT, B, K, MSE, DQ>(p, u, v, m, lane, kc, tab, nz, acc, pol);
-        },
-        MSE, pol);
+    tc::rotate_tiles<K>(&tp.xmap, p.n, smem_tc, p.fault, [&](int64_t u, f32x2 (&v)[EPT / 2]) {
+        normalize<EPT>(v, p.c_hi, p.c_lo);
+        float m[UnitShape<B, K>::NB];
+        block_max<B, K>(v, m);
+        quantize_values<FMT, B, K, MSE, DQ>(p, u, v, m, lane, kc, tab, nz, acc, pol);
+    });
     if constexpr (MSE) {
-        cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
-        finish_partials(p.partials, p.done, p.n, p.terms);
+        cta_partials<tc::THREADS>(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
+        finish_partials<tc::THREADS>(p.partials, p.done, p.n, p.terms);
     }
 }
 
@@ -368,15 +364,15 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_tc_kernel(QuantParams p)
 // normalisation y = fp32(s / sqrt(K)) rounds monotonically in s, so the
 // maximum is normalised once, after the maximum of the raw sums.
 template <int K>
-__global__ void __launch_bounds__(kThreads, 2) amax_tc_kernel(AmaxParams p)
+__global__ void __launch_bounds__(tc::THREADS, 3) amax_tc_kernel(const __grid_constant__ TcAmaxParams tp)
 {
+    const AmaxParams& p = tp.p;
     pdl_wait();
     pdl_release();
     extern __shared__ __align__(128) uint8_t smem_tc[];
     float mx = 0.0f;
-    tc::rotate_tiles<K>(
-        p.x, p.n, smem_tc, p.fault,
-        [&](int64_t, f32x2 (&v)[EPT / 2]) { mx = fmaxf(mx, pairs_absmax<EPT>(v)); }, false, 0);
+    tc::rotate_tiles<K>(&tp.xmap, p.n, smem_tc, p.fault,
+                        [&](int64_t, f32x2 (&v)[EPT / 2]) { mx = fmaxf(mx, pairs_absmax<EPT>(v)); });
     f32x2 m2[1] = {pk(mx, mx)};
     normalize<2>(m2, p.c_hi, p.c_lo);
     float a, b;
