@@ -12,16 +12,21 @@
 // operands [rows][K] row-major with blocks of b along K (fp4q_quantize_mma's
 // codes and MMA-layout scales).
 //
-// One CTA computes one 128 x 128 tile of Y, walking K in tiles of 256
-// elements (128 bytes of codes per row) through a ring of NSTAGE stages:
+// A persistent grid (one CTA per SM) walks the 128 x 128 tiles of Y; each
+// tile walks K in stages of 256 elements (128 bytes of codes per row) through
+// a ring of NSTAGE shared-memory stages:
 //   warp 0, one thread: TMA loads of the A and B code tiles (128-byte swizzle,
 //     straight into the layout the MMA reads) and bulk copies of the scale
 //     atoms, completing on the stage's `full` mbarrier;
 //   warp 1: allocates tensor memory; one thread copies each stage's scale
-//     atoms into tensor memory (tcgen05.cp) and issues the MMAs, then
-//     releases the stage through its `empty` mbarrier (tcgen05.commit);
+//     atoms into tensor memory (tcgen05.cp) and issues the MMAs into one of
+//     two accumulator buffers (alternating tile by tile), releasing the stage
+//     through its `empty` mbarrier (tcgen05.commit) and, after a tile's last
+//     stage, the buffer through `afull`;
 //   warps 2-5: the epilogue, each reading its 32 accumulator lanes
-//     (tcgen05.ld), scaling by G_A G_B and storing fp32 rows of Y.
+//     (tcgen05.ld), handing the buffer back (`aempty`), scaling by G_A G_B and
+//     storing fp32 rows of Y -- while the MMAs of the next tile run into the
+//     other buffer.
 // Every wait is bounded; a wait that runs out records the library's fault word
 // and the CTA stops its work and returns.
 #include <cuda.h>
@@ -42,10 +47,11 @@ constexpr int B_BYTES = BN * BKB;           // 16 KiB
 constexpr int SF_BYTES = 4 * 512;           // at most 4 scale atoms per operand per stage
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;   // 36 KiB
 constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 256;
-constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;         // accumulator 128 columns + scale ring 4 x 32
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 512;         // two 128-column accumulators + the scale ring, 4 x 32
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 128;
+constexpr uint32_t SF_COL = 2 * BN;
 constexpr uint32_t kMaxPolls = 1u << 24;
 
 struct Params {
@@ -146,17 +152,26 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_gemm_kernel(const __grid_const
     extern __shared__ __align__(1024) uint8_t smem_g[];
     const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_g);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const uint32_t bars = base + NSTAGE * STAGE_BYTES;      // full[NSTAGE], empty[NSTAGE], acc
-    const uint32_t full0 = bars, empty0 = bars + 8u * NSTAGE, acc_bar = bars + 16u * NSTAGE;
-    const uint32_t slot = acc_bar + 8u;
+    const uint32_t bars = base + NSTAGE * STAGE_BYTES;
+    const uint32_t full0 = bars, empty0 = full0 + 8u * NSTAGE;
+    const uint32_t afull0 = empty0 + 8u * NSTAGE, aempty0 = afull0 + 16u;   // 2 accumulator buffers
+    const uint32_t slot = aempty0 + 16u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int64_t m0 = (int64_t)blockIdx.y * BM, n0 = (int64_t)blockIdx.x * BN;
-    const int64_t kt_n = (p.k + BK - 1) / BK;              // stages of K (the last may be partial)
+    const int64_t tiles_n = (p.n + BN - 1) / BN;
+    const int64_t n_tiles = ((p.m + BM - 1) / BM) * tiles_n;
+    const int64_t kt_n = (p.k + BK - 1) / BK;              // stages of K per tile (the last may be partial)
     const int apk = p.nvfp4 ? 4 : 2;                         // scale atoms per full stage per operand
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2 * NSTAGE + 1; ++i) tc::mbar_init(bars + 8u * (uint32_t)i, 1u);
+        for (int i = 0; i < NSTAGE; ++i) {
+            tc::mbar_init(full0 + 8u * i, 1u);
+            tc::mbar_init(empty0 + 8u * i, 1u);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(afull0 + 8u * i, 1u);
+            tc::mbar_init(aempty0 + 8u * i, (uint32_t)EPI_WARPS);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) tc::tmem_alloc(slot, TMEM_COLS);
@@ -167,86 +182,112 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_gemm_kernel(const __grid_const
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(tmem) : "r"(slot) : "memory");
 
     if (warp == 0 && lane == 0) {
-        // ---- producer
-        for (int64_t kt = 0; kt < kt_n; ++kt) {
-            const int s = (int)(kt % NSTAGE);
-            const int64_t use = kt / NSTAGE;
-            if (use > 0 && !wait_phase(empty0 + 8u * s, (uint32_t)((use - 1) & 1), p.fault)) break;
-            const int steps = (int)((p.k - kt * BK) >= BK ? 4 : (p.k - kt * BK) / 64);
-            const int64_t atom0 = kt * apk;
-            int natoms = p.nvfp4 ? steps : (steps + 1) / 2;
-            if (atom0 + natoms > p.sf_kt) natoms = (int)(p.sf_kt - atom0);
-            const uint32_t st = base + (uint32_t)(s * STAGE_BYTES);
-            const uint32_t fb = full0 + 8u * s;
-            mbar_expect_tx(fb, (uint32_t)(A_BYTES + B_BYTES + 2 * natoms * 512));
-            tma_load_2d(st, &p.ta, (int)(kt * BKB), (int)m0, fb);
-            tma_load_2d(st + A_BYTES, &p.tb, (int)(kt * BKB), (int)n0, fb);
-            const uint8_t* sa = p.sfa + (((m0 >> 7) * p.sf_kt + atom0) << 9);
-            const uint8_t* sb = p.sfb + (((n0 >> 7) * p.sf_kt + atom0) << 9);
-            bulk_load(st + A_BYTES + B_BYTES, sa, (uint32_t)natoms * 512u, fb);
-            bulk_load(st + A_BYTES + B_BYTES + SF_BYTES, sb, (uint32_t)natoms * 512u, fb);
+        // ---- producer: the (tile, k-stage) sequence of this CTA through the ring
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.ta)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tb)) : "memory");
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            const int64_t m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+            for (int64_t kt = 0; kt < kt_n; ++kt, ++g) {
+                const int s = (int)(g % NSTAGE);
+                if (g >= NSTAGE && !wait_phase(empty0 + 8u * s, (uint32_t)(((g / NSTAGE) - 1) & 1), p.fault)) {
+                    ok = false;
+                    break;
+                }
+                const int steps = (int)((p.k - kt * BK) >= BK ? 4 : (p.k - kt * BK) / 64);
+                const int64_t atom0 = kt * apk;
+                int natoms = p.nvfp4 ? steps : (steps + 1) / 2;
+                if (atom0 + natoms > p.sf_kt) natoms = (int)(p.sf_kt - atom0);
+                const uint32_t st = base + (uint32_t)(s * STAGE_BYTES);
+                const uint32_t fb = full0 + 8u * s;
+                mbar_expect_tx(fb, (uint32_t)(A_BYTES + B_BYTES + 2 * natoms * 512));
+                tma_load_2d(st, &p.ta, (int)(kt * BKB), (int)m0, fb);
+                tma_load_2d(st + A_BYTES, &p.tb, (int)(kt * BKB), (int)n0, fb);
+                const uint8_t* sa = p.sfa + (((m0 >> 7) * p.sf_kt + atom0) << 9);
+                const uint8_t* sb = p.sfb + (((n0 >> 7) * p.sf_kt + atom0) << 9);
+                bulk_load(st + A_BYTES + B_BYTES, sa, (uint32_t)natoms * 512u, fb);
+                bulk_load(st + A_BYTES + B_BYTES + SF_BYTES, sb, (uint32_t)natoms * 512u, fb);
+            }
         }
     } else if (warp == 1 && lane == 0) {
-        // ---- scale copies and MMAs
+        // ---- scale copies and MMAs, one accumulator buffer per tile, alternating
+        int64_t g = 0, j = 0;
         bool ok = true;
-        for (int64_t kt = 0; kt < kt_n && ok; ++kt) {
-            const int s = (int)(kt % NSTAGE);
-            if (!wait_phase(full0 + 8u * s, (uint32_t)((kt / NSTAGE) & 1), p.fault)) {
-                ok = false;
-                break;
-            }
-            tc::tc_fence_after();
-            const int steps = (int)((p.k - kt * BK) >= BK ? 4 : (p.k - kt * BK) / 64);
-            const int64_t atom0 = kt * apk;
-            int natoms = p.nvfp4 ? steps : (steps + 1) / 2;
-            if (atom0 + natoms > p.sf_kt) natoms = (int)(p.sf_kt - atom0);
-            const uint32_t st = base + (uint32_t)(s * STAGE_BYTES);
-            const uint32_t sf_a = tmem + SF_COL + 32u * (uint32_t)s;     // 4 columns per atom
-            const uint32_t sf_b = sf_a + 16u;
-            for (int a = 0; a < natoms; ++a) {
-                tmem_cp_atom(sf_a + 4u * a, atom_desc(st + A_BYTES + B_BYTES + 512u * a));
-                tmem_cp_atom(sf_b + 4u * a, atom_desc(st + A_BYTES + B_BYTES + SF_BYTES + 512u * a));
-            }
-            for (int kk = 0; kk < steps; ++kk) {
-                const uint64_t da = sw128_desc(st + 32u * kk);
-                const uint64_t db = sw128_desc(st + A_BYTES + 32u * kk);
-                const bool acc = kt > 0 || kk > 0;
-                if (p.nvfp4) {
-                    mma_nvfp4(tmem + ACC_COL, da, db, bs_idesc(true, 0), sf_a + 4u * kk, sf_b + 4u * kk, acc);
-                } else {
-                    const uint32_t id = 2u * (uint32_t)(kk & 1);
-                    const uint32_t col = 4u * (uint32_t)(kk >> 1);
-                    mma_mxfp4(tmem + ACC_COL, da, db, bs_idesc(false, id), (sf_a + col) | (id << 30),
-                              (sf_b + col) | (id << 30), acc);
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++j) {
+            const int ab = (int)(j & 1);
+            if (j >= 2 && !wait_phase(aempty0 + 8u * ab, (uint32_t)(((j >> 1) - 1) & 1), p.fault)) break;
+            const uint32_t acc_col = tmem + ACC_COL + (uint32_t)(ab * BN);
+            for (int64_t kt = 0; kt < kt_n; ++kt, ++g) {
+                const int s = (int)(g % NSTAGE);
+                if (!wait_phase(full0 + 8u * s, (uint32_t)((g / NSTAGE) & 1), p.fault)) {
+                    ok = false;
+                    break;
                 }
+                tc::tc_fence_after();
+                const int steps = (int)((p.k - kt * BK) >= BK ? 4 : (p.k - kt * BK) / 64);
+                const int64_t atom0 = kt * apk;
+                int natoms = p.nvfp4 ? steps : (steps + 1) / 2;
+                if (atom0 + natoms > p.sf_kt) natoms = (int)(p.sf_kt - atom0);
+                const uint32_t st = base + (uint32_t)(s * STAGE_BYTES);
+                const uint32_t sf_a = tmem + SF_COL + 32u * (uint32_t)s;     // 4 columns per atom
+                const uint32_t sf_b = sf_a + 16u;
+                for (int a = 0; a < natoms; ++a) {
+                    tmem_cp_atom(sf_a + 4u * a, atom_desc(st + A_BYTES + B_BYTES + 512u * a));
+                    tmem_cp_atom(sf_b + 4u * a, atom_desc(st + A_BYTES + B_BYTES + SF_BYTES + 512u * a));
+                }
+                for (int kk = 0; kk < steps; ++kk) {
+                    const uint64_t da = sw128_desc(st + 32u * kk);
+                    const uint64_t db = sw128_desc(st + A_BYTES + 32u * kk);
+                    const bool acc = kt > 0 || kk > 0;
+                    if (p.nvfp4) {
+                        mma_nvfp4(acc_col, da, db, bs_idesc(true, 0), sf_a + 4u * kk, sf_b + 4u * kk, acc);
+                    } else {
+                        const uint32_t id = 2u * (uint32_t)(kk & 1);
+                        const uint32_t col = 4u * (uint32_t)(kk >> 1);
+                        mma_mxfp4(acc_col, da, db, bs_idesc(false, id), (sf_a + col) | (id << 30),
+                                  (sf_b + col) | (id << 30), acc);
+                    }
+                }
+                tc::mma_commit(empty0 + 8u * s);        // the stage (smem and its scale columns) is free again
             }
-            tc::mma_commit(empty0 + 8u * s);            // the stage (smem and its scale columns) is free again
+            if (ok) tc::mma_commit(afull0 + 8u * ab);   // the tile's accumulator is complete
         }
-        if (ok) tc::mma_commit(acc_bar);
     } else if (warp >= 2) {
         // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31
         const int q = warp & 3;
-        bool done = wait_phase(acc_bar, 0u, p.fault);
-        const bool have = __all_sync(0xffffffffu, done) && kt_n > 0;
-        if (have) {
+        const float g = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f);
+        int64_t j = 0;
+        for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++j) {
+            const int ab = (int)(j & 1);
+            const bool done = wait_phase(afull0 + 8u * ab, (uint32_t)((j >> 1) & 1), p.fault);
+            if (!__all_sync(0xffffffffu, done)) break;
             tc::tc_fence_after();
-            const float g = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f);
+            const int64_t m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
             const int64_t r = m0 + 32 * q + lane;
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
-                tc::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + ACC_COL + 32u * (uint32_t)c, v);
+                tc::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + ACC_COL + (uint32_t)(ab * BN) + 32u * (uint32_t)c,
+                              v);
+                if (c == BN / 32 - 1) {
+                    // every column of this warp's lanes is in registers: the buffer may be refilled
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(aempty0 + 8u * ab);
+                }
                 const int64_t c0 = n0 + 32 * c;
                 if (r < p.m && c0 < p.n) {
                     float* dst = p.y + r * p.n + c0;
                     if (c0 + 32 <= p.n && (p.n & 3) == 0) {
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            stg128(dst + j, __float_as_uint(__fmul_rn(__uint_as_float(v[j]), g)),
-                                   __float_as_uint(__fmul_rn(__uint_as_float(v[j + 1]), g)),
-                                   __float_as_uint(__fmul_rn(__uint_as_float(v[j + 2]), g)),
-                                   __float_as_uint(__fmul_rn(__uint_as_float(v[j + 3]), g)));
+                        for (int jj = 0; jj < 32; jj += 4)
+                            stg128(dst + jj, __float_as_uint(__fmul_rn(__uint_as_float(v[jj]), g)),
+                                   __float_as_uint(__fmul_rn(__uint_as_float(v[jj + 1]), g)),
+                                   __float_as_uint(__fmul_rn(__uint_as_float(v[jj + 2]), g)),
+                                   __float_as_uint(__fmul_rn(__uint_as_float(v[jj + 3]), g)));
                     } else {
-                        for (int j = 0; j < 32 && c0 + j < p.n; ++j) dst[j] = __fmul_rn(__uint_as_float(v[j]), g);
+                        for (int jj = 0; jj < 32 && c0 + jj < p.n; ++jj)
+                            dst[jj] = __fmul_rn(__uint_as_float(v[jj]), g);
                     }
                 }
             }
@@ -308,17 +349,8 @@ extern "C" int fp4q_gemm(const uint8_t* codes_a, const uint8_t* scales_a, const 
     p.nvfp4 = fmt == FP4Q_SCALE_UE4M3;
     p.fault = device_fault_word();
     if (!p.fault) return FP4Q_ERR_CUDA;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(gemm::fp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::SMEM_BYTES) != cudaSuccess)
-            return FP4Q_ERR_CUDA;
-        attr_set[dev] = true;
-    }
-    const dim3 grid((unsigned)((n + gemm::BN - 1) / gemm::BN), (unsigned)((m + gemm::BM - 1) / gemm::BM));
-    if (grid.y > 65535u) return FP4Q_ERR_SHAPE;
+    const int64_t tiles = ((m + gemm::BM - 1) / gemm::BM) * ((n + gemm::BN - 1) / gemm::BN);
+    const int grid = grid_for((const void*)gemm::fp4_gemm_kernel, gemm::SMEM_BYTES, tiles, gemm::THREADS);
     gemm::fp4_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
 }

@@ -115,22 +115,26 @@ namespace {
 template <int K>
 cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
+    // the rotation on the tensor cores, 4096-element tiles through a TMA ring of
+    // 32-element rows; a tensor whose size is an odd multiple of 16 rotates with
+    // the butterfly kernel below
     if constexpr (K == 16 || K == 32) {
-        // the rotation on the tensor cores: 4096-element tiles through a TMA ring
-        TcAmaxParams tp;
-        memset(&tp, 0, sizeof(tp));
-        tp.p = p;
-        tp.p.fault = device_fault_word();
-        if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
-        if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
-                                  tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
-            return cudaErrorInvalidValue;
-        auto kern = amax_tc_kernel<K>;
-        const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
-        const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, tiles, tc::THREADS);
-        if (pdl) return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
-        kern<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(tp);
-        return cudaGetLastError();
+        if (p.n % 32 == 0) {
+            TcAmaxParams tp;
+            memset(&tp, 0, sizeof(tp));
+            tp.p = p;
+            tp.p.fault = device_fault_word();
+            if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
+            if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
+                                      tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+            auto kern = amax_tc_kernel<K>;
+            const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
+            const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, tiles, tc::THREADS);
+            if (pdl) return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
+            kern<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(tp);
+            return cudaGetLastError();
+        }
     }
     auto kern = amax_kernel<K>;
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));

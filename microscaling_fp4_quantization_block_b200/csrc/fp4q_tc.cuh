@@ -17,12 +17,14 @@
 // holds the 32 rotated values of "its" row: the same 32-element unit the
 // quantizer works on, with no shuffles.
 //
-// Warp-specialised pipeline (a CTA of 4 consumer warps and 1 control warp):
-//   control warp, lane 0: TMA loads of 4096-element tiles (a 2-D tensor map
-//     of 64-byte rows with the 64-byte swizzle, which is the K-major layout
+// Warp-specialised pipeline (a CTA of 4 consumer warps, a producer warp and an
+// MMA warp; the two single-thread roles sit in different warps so that a
+// blocking mbarrier probe in one never stalls the other):
+//   producer warp, one thread: TMA loads of 4096-element tiles (a 2-D tensor
+//     map of 64-byte rows with the 64-byte swizzle, which is the K-major layout
 //     the MMA reads) into a ring of NSTAGE shared-memory stages, completing on
 //     the stage's `full` mbarrier;
-//   control warp, lane 1: per tile, the two K = 16 MMAs into one of NBUF TMEM
+//   MMA warp, one thread: per tile, the two K = 16 MMAs into one of NBUF TMEM
 //     accumulator buffers, then tcgen05.commit on the stage's `empty` barrier
 //     (the stage may be refilled) and the buffer's `tfull` barrier;
 //   consumer warps: per tile, wait for `tfull`, tcgen05.ld their 32 lanes,
@@ -46,7 +48,9 @@ constexpr int STAGE_BYTES = ROWS * KR * 2;      // 8 KiB of bf16
 constexpr int NSTAGE = 6;                       // shared-memory ring stages
 constexpr int NBUF = 4;                         // TMEM accumulator buffers of 32 columns
 constexpr int CONSUMER_WARPS = 4;
-constexpr int THREADS = 32 * (CONSUMER_WARPS + 1);
+constexpr int PRODUCER_WARP = CONSUMER_WARPS;   // TMA loads
+constexpr int MMA_WARP = CONSUMER_WARPS + 1;    // TMEM allocation and the MMAs
+constexpr int THREADS = 32 * (CONSUMER_WARPS + 2);
 constexpr int TMEM_COLS = NBUF * KR;            // 128 (a power of two >= 32)
 constexpr int B_BYTES = KR * KR * 2;            // the rotation matrix, 2 KiB
 // dynamic shared memory: 1 KiB of slack to align the swizzled buffers to 1 KiB,
@@ -238,7 +242,7 @@ __device__ __forceinline__ void rotate_tiles(const void* xmap, int64_t n, uint8_
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == CONSUMER_WARPS) tmem_alloc(slot, TMEM_COLS);
+    if (warp == MMA_WARP) tmem_alloc(slot, TMEM_COLS);
     fence_proxy_async_smem();                                    // the rotation matrix, for the MMA
     tc_fence_before();
     __syncthreads();
@@ -249,7 +253,7 @@ __device__ __forceinline__ void rotate_tiles(const void* xmap, int64_t n, uint8_
     const int64_t n_tiles = (n + TILE_ELEMS - 1) / TILE_ELEMS;
     const int64_t first = blockIdx.x, stride = gridDim.x;
 
-    if (warp == CONSUMER_WARPS) {
+    if (warp == PRODUCER_WARP) {
         if (lane == 0) {
             // ---- TMA producer
             int64_t i = 0;
@@ -259,7 +263,10 @@ __device__ __forceinline__ void rotate_tiles(const void* xmap, int64_t n, uint8_
                 mbar_expect_tx(full0 + 8u * s, (uint32_t)STAGE_BYTES);
                 tma_load_2d(ring + (uint32_t)(s * STAGE_BYTES), xmap, 0, (int)(t * ROWS), full0 + 8u * s);
             }
-        } else if (lane == 1) {
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        if (lane == 0) {
             // ---- MMA issuer
             int64_t i = 0;
             for (int64_t t = first; t < n_tiles; t += stride, ++i) {
@@ -301,7 +308,7 @@ __device__ __forceinline__ void rotate_tiles(const void* xmap, int64_t n, uint8_
     // role gave up), so TMEM can be released
     tc_fence_before();
     __syncthreads();
-    if (warp == CONSUMER_WARPS) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
             "orc_nearest_rank": (I64, [ctypes.c_double, I64]),
             "orc_fp4_gemm": (I, [P, P, F, I64, P, P, F, I64, I64, I, I, P]),
             "orc_outlier_stats_bf16": (I, [P, I64, I64, ctypes.c_double, P, P]),
+            "orc_global_scale_search_f32": (I, [P, I64, I64, I, I, I, I, I, P, P, P, P]),
+            "orc_global_scale_search_bf16": (I, [P, I64, I64, I, I, I, I, I, P, P, P, P]),
             "orc_block_mse_f32": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
             "orc_block_mse_bf16": (I, [P, P, P, F, I64, I64, I, I, I, P, P]),
         }
@@ -234,6 +236,25 @@ def quantize_search(x, fmt: int, block: int, rot: int = 0, gmode: int = G_NONE, 
     _check(fn(_ptr(x), rows, cols, fmt, block, rot, gmode, below, above, _ptr(g), _ptr(codes), _ptr(scales)),
            "quantize_search")
     return codes, scales, float(g[0])
+
+
+def global_scale_search(x, fmt: int, block: int, rot: int = 0, below: int = 4, above: int = 4):
+    """MSE-optimised per-tensor scale: candidates G_j = fp32(G0 (16 + j) / 16),
+    j in [-below, above], the max rule for the block scales under each.
+    Returns ``(codes, scales, G*, errs)`` with errs[j + below] the candidate's
+    per-tensor MSE (fp64)."""
+    x = np.ascontiguousarray(x)
+    if x.ndim != 2:
+        raise ValueError("expected a 2-D array")
+    rows, cols = x.shape
+    codes = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // block if block else 0), np.uint8)
+    g = np.zeros(1, np.float32)
+    errs = np.full(below + above + 1, np.nan, np.float64)
+    fn = lib().orc_global_scale_search_bf16 if x.dtype == np.uint16 else lib().orc_global_scale_search_f32
+    _check(fn(_ptr(x), rows, cols, fmt, block, rot, below, above, _ptr(g), _ptr(errs), _ptr(codes), _ptr(scales)),
+           "global_scale_search")
+    return codes, scales, float(g[0]), errs
 
 
 def quantize_with_scales(x, scales, G: float, fmt: int, block: int, rot: int = 0) -> np.ndarray:

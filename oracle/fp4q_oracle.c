@@ -708,3 +708,83 @@ int orc_fp4_gemm(const uint8_t* codes_a, const uint8_t* scales_a, float ga, int6
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MSE-optimised per-tensor scale ([B] s3.2, MR-GPTQ item 2: the global      */
+/* scale is optimised together with the group scales, instead of being set  */
+/* by the max rule alone).  The pages give no procedure; the reading taken   */
+/* here: the candidates are G_j = fp32(G0 (16 + j) / 16), j in [-below,     */
+/* above] (below <= 8, above <= 15: from half to almost twice the max-rule   */
+/* scale G0 = amax / 2688, 1 for an all-zero tensor), tried in the order     */
+/* j = 0, 1, -1, 2, -2, ...; under each, the block scales follow the max     */
+/* rule and the error is the exact (fp64) sum of squared errors over the     */
+/* whole tensor; a candidate replaces the best only when its error is        */
+/* strictly smaller, so ties keep the earlier one and G0 wins every tie.     */
+/* UE4M3 and UE5M3 only (E8M0 has no per-tensor scale).  Writes G* to        */
+/* *gscale, the error of candidate j (divided by n) to errs[j + below], and  */
+/* the codes and scale bytes under G*.                                       */
+
+int orc_global_scale_search_f32(const float* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                int below, int above, float* gscale, double* errs, uint8_t* codes,
+                                uint8_t* scales)
+{
+    int st = check_layout(rows, cols, fmt, block, rot);
+    if (st) return st;
+    if (fmt == ORC_E8M0) return ORC_EARG;
+    if (below < 0 || below > 8 || above < 0 || above > 15) return ORC_EARG;
+    const int64_t n = rows * cols;
+    float* y = domain_values(x, n, rot);
+    if (!y) return ORC_ENOMEM;
+    const float g0 = orc_global_scale_from_amax(orc_tensor_amax(y, n));
+    free(y);
+    uint8_t* c = (uint8_t*)malloc((size_t)(n / 2 > 0 ? n / 2 : 1));
+    uint8_t* s = (uint8_t*)malloc((size_t)(n / block > 0 ? n / block : 1));
+    if (!c || !s) {
+        free(c);
+        free(s);
+        return ORC_ENOMEM;
+    }
+    double terms[4];
+    int best = 0, have = 0;
+    double best_err = 0.0;
+    const int span = below > above ? below : above;
+    for (int t = 0; t <= 2 * span; ++t) {
+        /* t = 0, 1, 2, 3, 4 ... -> j = 0, 1, -1, 2, -2, ... */
+        const int j = t == 0 ? 0 : ((t & 1) ? (t + 1) / 2 : -(t / 2));
+        if (j > above || -j > below) continue;
+        float G = (float)((double)g0 * (double)(16 + j) / 16.0);
+        st = orc_quantize_f32(x, rows, cols, fmt, block, rot, ORC_G_GIVEN, &G, c, s);
+        if (st) break;
+        st = orc_block_mse_f32(x, c, s, G, rows, cols, fmt, block, rot, NULL, terms);
+        if (st) break;
+        errs[j + below] = terms[0];
+        if (!have || terms[0] < best_err) {
+            best = j;
+            best_err = terms[0];
+            have = 1;
+        }
+    }
+    if (!st) {
+        float G = (float)((double)g0 * (double)(16 + best) / 16.0);
+        *gscale = G;
+        st = orc_quantize_f32(x, rows, cols, fmt, block, rot, ORC_G_GIVEN, &G, codes, scales);
+    }
+    free(c);
+    free(s);
+    return st;
+}
+
+int orc_global_scale_search_bf16(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                 int below, int above, float* gscale, double* errs, uint8_t* codes,
+                                 uint8_t* scales)
+{
+    if (rows < 0 || cols < 0) return ORC_ESHAPE;
+    const int64_t n = rows * cols;
+    float* xf = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
+    if (!xf) return ORC_ENOMEM;
+    orc_bf16_to_f32_array(x, n, xf);
+    int st = orc_global_scale_search_f32(xf, rows, cols, fmt, block, rot, below, above, gscale, errs, codes,
+                                         scales);
+    free(xf);
+    return st;
+}

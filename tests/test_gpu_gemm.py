@@ -149,3 +149,24 @@ def test_gemm_edge_cases(fq):
     with pytest.raises(Exception):
         fq.fp4q_quantize_mma(x, U4, 32)
     assert fq.fp4q_device_fault() == 0
+
+
+@pytest.mark.parametrize("fmt", [E8, U4])
+@pytest.mark.parametrize("m,n,k", [(4096, 1024, 256), (8192, 2048, 128)])
+def test_persistent_many_tiles(fq, fmt, m, n, k):
+    """More 128 x 128 tiles than CTAs (256 and 1024 tiles on 148 SMs): both
+    accumulator buffers and every barrier phase are reused; lossless operands,
+    so every element of Y is checked exactly."""
+    rng = np.random.default_rng(m + n + k + fmt)
+    a, b = _lossless(m, k, rng, fmt), _lossless(n, k, rng, fmt)
+    ca, sa, _, sa_rm = _operands(fq, a, fmt, "none")
+    cb, sb, _, sb_rm = _operands(fq, b, fmt, "none")
+    y = fq.fp4q_gemm(ca, sa, None, cb, sb, None, fmt)
+    torch.cuda.synchronize()
+    want = a.cuda().double() @ b.cuda().double().T          # exact: the operands are lossless
+    assert torch.equal(y.double(), want)
+    block = 16 if fmt == U4 else 32
+    rows = np.r_[0:3, m - 3:m]
+    sub = oracle.fp4_gemm(ca.cpu().numpy()[rows], sa_rm[rows], 1.0, cb.cpu().numpy(), sb_rm, 1.0, k, fmt, block)
+    assert np.array_equal(sub, want.cpu().numpy()[rows])
+    assert fq.fp4q_device_fault() == 0
