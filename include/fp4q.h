@@ -316,6 +316,26 @@ FP4Q_API int fp4q_block_mse_noalloc(const void* x, const uint8_t* codes, const u
 FP4Q_API int fp4q_e2m1_encode_f32(const float* r, int64_t n, uint8_t* packed, void* stream);
 FP4Q_API int fp4q_scale_encode_f32(const float* s, int64_t n, int fmt, uint8_t* codes, void* stream);
 
+/* MSE-optimised per-tensor scale ("Bridging the Gap", s3.2, MR-GPTQ item 2:
+ * the global scale optimised together with the group scales).  Candidates
+ * G_j = fp32(G0 * (16 + j) / 16) for j in [-below, above] (0 <= below <= 8,
+ * 0 <= above <= 15), G0 = amax / 2688 of the (rotated) tensor (1 when it is
+ * all zero), tried in the order j = 0, 1, -1, 2, -2, ...; under each, block
+ * scales by the max rule; the candidate whose total squared error is
+ * strictly smallest is kept, so G0 wins every tie.  Writes G* to gscale[0]
+ * (device float) and, if errors != NULL, each candidate's per-tensor MSE to
+ * errors[j + below] (device doubles).  The codes for G* are then
+ * fp4q_quantize(..., FP4Q_GLOBAL_GIVEN, gscale).  fmt UE4M3 or UE5M3 (E8M0
+ * has no per-tensor scale: FP4Q_ERR_UNSUPPORTED); block and rot as
+ * fp4q_quantize.  workspace: device, 16-byte aligned, at least
+ * fp4q_global_scale_search_workspace_size() bytes, no initial contents
+ * required (the call clears what it needs).  One pass over x for the
+ * maximum and one for all candidates; enqueued on `stream`. */
+FP4Q_API int fp4q_global_scale_search(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot,
+                                      int below, int above, float* gscale, double* errors, void* workspace,
+                                      size_t ws_bytes, void* stream);
+FP4Q_API size_t fp4q_global_scale_search_workspace_size(void);
+
 /* fp4q_quantize with the scale bytes written in the layout the block-scaled
  * tensor-core MMA reads them from (the operand layout of fp4q_gemm), for the
  * two formats that MMA takes: MXFP4 (E8M0, block 32) and NVFP4 (UE4M3, block

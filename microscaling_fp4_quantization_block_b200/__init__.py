@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
         "fp4q_quantize_mma": (I, [P, I64, I64, I, I, I, I, P, P, P, P]),
         "fp4q_mma_scales_size": (ctypes.c_size_t, [I64, I64, I]),
         "fp4q_gemm": (I, [P, P, P, I64, P, P, P, I64, I64, I, P, P]),
+        "fp4q_global_scale_search": (I, [P, I64, I64, I, I, I, I, I, P, P, P, ctypes.c_size_t, P]),
+        "fp4q_global_scale_search_workspace_size": (ctypes.c_size_t, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -156,6 +158,30 @@ def fp4q_quantize(x: torch.Tensor, fmt, block: int, rot: int = 0, gmode="none",
                             _ptr(gscale), _stream(stream))
     _check(st, "fp4q_quantize")
     return codes, scales, gscale
+
+
+def fp4q_global_scale_search(x: torch.Tensor, fmt, block: int, rot: int = 0, below: int = 8, above: int = 15,
+                             gscale: Optional[torch.Tensor] = None, errors: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None
+                             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MSE-optimised per-tensor scale: returns (gscale [1], errors [below + above + 1])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    _need_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    dev = x.device
+    if gscale is None:
+        gscale = torch.empty((1,), dtype=torch.float32, device=dev)
+    if errors is None:
+        errors = torch.empty((below + above + 1,), dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.empty((lib().fp4q_global_scale_search_workspace_size(),), dtype=torch.uint8, device=dev)
+    _need_cuda(gscale, errors, workspace)
+    st = lib().fp4q_global_scale_search(_ptr(x), rows, cols, _fmt(fmt), block, rot, below, above, _ptr(gscale),
+                                        _ptr(errors), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "fp4q_global_scale_search")
+    return gscale, errors
 
 
 def fp4q_mma_scales_size(rows: int, cols: int, block: int) -> int:

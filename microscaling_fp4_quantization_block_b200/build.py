@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libfp4q.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 SOURCES = ["fp4q_api.cu", "fp4q_quantize.cu", "fp4q_quantize_e8m0.cu", "fp4q_quantize_ue4m3.cu",
-           "fp4q_quantize_ue5m3.cu", "fp4q_search.cu", "fp4q_stats.cu", "fp4q_dequantize.cu", "fp4q_gemm.cu"]
+           "fp4q_quantize_ue5m3.cu", "fp4q_search.cu", "fp4q_stats.cu", "fp4q_dequantize.cu", "fp4q_gemm.cu", "fp4q_gscale.cu"]
 HEADERS = ["fp4q_device.cuh", "fp4q_kernels.cuh", "fp4q_launch.h", "fp4q_quantize_impl.cuh", "fp4q_tc.cuh"]
 
 NVCC_FLAGS = [

@@ -265,6 +265,41 @@ int fp4q_quantize(const void* x, int64_t rows, int64_t cols, int fmt, int block,
     return quantize_impl(x, rows, cols, fmt, block, rot, gmode, codes, scales, gscale, false, 0, 0, stream);
 }
 
+size_t fp4q_global_scale_search_workspace_size(void) { return gscale_workspace_bytes(); }
+
+int fp4q_global_scale_search(const void* x, int64_t rows, int64_t cols, int fmt, int block, int rot, int below,
+                             int above, float* gscale, double* errors, void* workspace, size_t ws_bytes,
+                             void* stream)
+{
+    int64_t n = 0;
+    int st = check_shape(rows, cols, fmt, block, rot, &n);
+    if (st) return st;
+    if (fmt == FP4Q_SCALE_E8M0) return FP4Q_ERR_UNSUPPORTED;
+    if (below < 0 || below > 8 || above < 0 || above > 15) return FP4Q_ERR_UNSUPPORTED;
+    if (!gscale || !workspace) return FP4Q_ERR_NULL;
+    if (!aligned(gscale, 4) || !aligned(workspace, 16) || (errors && !aligned(errors, 8))) return FP4Q_ERR_ALIGN;
+    if (ws_bytes < gscale_workspace_bytes()) return FP4Q_ERR_WORKSPACE;
+    if (n > 0 && !x) return FP4Q_ERR_NULL;
+    if (n > 0 && !aligned(x, 32)) return FP4Q_ERR_ALIGN;
+    cudaStream_t s = as_stream(stream);
+    if (n == 0) {
+        // an empty tensor: G0 = 1 is the only sensible scale; every candidate's error is 0
+        if (errors && cudaMemsetAsync(errors, 0, (size_t)(below + above + 1) * sizeof(double), s) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        if (cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 16, 0, 4, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+        global_scale_kernel<<<1, 1, 0, s>>>(static_cast<const float*>(workspace) + 4, gscale);
+        return cuda_status(cudaGetLastError());
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return FP4Q_ERR_CUDA;          // completion counter
+    cudaError_t e = enqueue_amax(x, n, rot, reinterpret_cast<float*>(ws + 16), s);  // the tensor maximum
+    if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+    float c_hi = 0.0f, c_lo = 0.0f;
+    rotation_constants(rot, &c_hi, &c_lo);
+    return cuda_status(launch_gscale_search(static_cast<const uint16_t*>(x), n, fmt, block, rot, c_hi, c_lo, below,
+                                            above, gscale, errors, workspace, s));
+}
+
 size_t fp4q_mma_scales_size(int64_t rows, int64_t cols, int block)
 {
     if (rows <= 0 || cols <= 0 || block <= 0) return 0;

@@ -53,6 +53,11 @@ cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, double p, float* stats,
                                  float* col_absmax, void* workspace, cudaStream_t s);
 cudaError_t launch_dequantize(int B, int K, bool f32out, const DequantParams& p, cudaStream_t s);
+// MSE-optimised per-tensor scale: reads the tensor maximum from workspace + 16
+// (written by the amax pass), counter at workspace + 0 (zero at launch).
+cudaError_t launch_gscale_search(const uint16_t* x, int64_t n, int fmt, int block, int rot, float c_hi, float c_lo,
+                                 int below, int above, float* gscale, double* errors, void* workspace, cudaStream_t s);
+size_t gscale_workspace_bytes();
 cudaError_t launch_block_mse(int B, int K, const MseParams& p, int* grid_out, cudaStream_t s);
 
 // Launch of a streaming kernel with programmatic dependent launch allowed: the

@@ -181,3 +181,20 @@ def test_gemm_and_mma_layout_reject_bad_arguments(fp4q):
     assert qm(A32, 4, 64, U4, 16, 0, 0, A32, A32 + 8, None, None) == -3
     assert qm(None, 0, 64, U4, 16, 0, 0, None, None, None, None) == 0
     assert L.fp4q_device_fault(None, 0) == -1
+
+
+def test_global_scale_search_rejects_bad_arguments(fp4q):
+    L = fp4q.lib()
+    ws = L.fp4q_global_scale_search_workspace_size()
+    assert ws >= 32 + 4096 * 24 * 8
+    g = L.fp4q_global_scale_search
+    assert g(A32, 4, 64, 0, 32, 0, 1, 1, A32, None, A32, ws, None) == -4       # E8M0: no per-tensor scale
+    assert g(A32, 4, 64, 1, 16, 0, 9, 1, A32, None, A32, ws, None) == -4       # below > 8
+    assert g(A32, 4, 64, 1, 16, 0, 1, 16, A32, None, A32, ws, None) == -4      # above > 15
+    assert g(A32, 4, 60, 1, 16, 0, 1, 1, A32, None, A32, ws, None) == -2
+    assert g(A32, 4, 64, 1, 16, 0, 1, 1, None, None, A32, ws, None) == -1
+    assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32, None, None, ws, None) == -1
+    assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32, None, A32, ws - 8, None) == -6
+    assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32 + 2, None, A32, ws, None) == -3
+    assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32, A32 + 4, A32, ws, None) == -3
+    assert g(A32 + 16, 4, 64, 1, 16, 0, 1, 1, A32, None, A32, ws, None) == -3
