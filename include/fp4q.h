@@ -376,11 +376,9 @@ FP4Q_API int fp4q_gemm(const uint8_t* codes_a, const uint8_t* scales_a, const fl
 FP4Q_API size_t fp4q_mma_scales_size(int64_t rows, int64_t cols, int block);
 
 /* The library's device fault word on the current device, read into
- * *fault_out: 0 normally; 1 once a kernel that rotates on the tensor cores
- * (rot 16 or 32 in fp4q_quantize, fp4q_quantize_mse,
- * fp4q_quantize_mse_dequantize and fp4q_tensor_amax[_accumulate]) gave up a
- * bounded wait for its matrix-multiply instructions instead of hanging; the
- * outputs of that call are then incomplete.  clear != 0 resets the word to 0
+ * *fault_out: 0 normally; 1 once a kernel on the tensor cores (fp4q_gemm)
+ * gave up a bounded wait for its copies or matrix-multiply instructions
+ * instead of hanging; the outputs of that call are then incomplete.  clear != 0 resets the word to 0
  * after reading it.  The pages have no counterpart: this is the library's own
  * failure report.  Unlike every other entry point this call synchronizes the
  * current device (it reads device memory).  FP4Q_ERR_NULL if fault_out is

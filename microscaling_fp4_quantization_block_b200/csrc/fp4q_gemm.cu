@@ -31,6 +31,9 @@
 // and the CTA stops its work and returns.
 #include <cuda.h>
 
+#include <mutex>
+
+#include "fp4q_device.cuh"
 #include "fp4q_launch.h"
 #include "fp4q_tc.cuh"
 #include "../../include/fp4q.h"
@@ -302,10 +305,41 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_gemm_kernel(const __grid_const
     }
 }
 
+// The driver's cuTensorMapEncodeTiled, fetched once at run time (the library
+// links the runtime only).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// The code tiles of an operand: [rows][k / 2] bytes, boxes of 128 rows x 128
+// bytes (one 128-byte swizzle row per K stage), 128-byte swizzle.
 bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k)
 {
-    return encode_tensor_map_2d(map, 1, codes, (uint64_t)(k / 2), (uint64_t)rows, (uint64_t)(k / 2), BKB, BM,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
+    EncodeTiledFn enc = encode_fn();
+    const uint64_t inner = (uint64_t)(k / 2);
+    if (!enc || rows <= 0 || inner == 0) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)inner};
+    const cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)BM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace gemm

@@ -463,7 +463,6 @@ struct QuantParams {
     float* gdst;           // G from the tensor maximum: *gsrc is that maximum, G is written here
     uint16_t* y;           // fused MSE with dequantized output: n bf16 values
     int below, above;      // scale search: codes tried below / above the max-rule code
-    unsigned int* fault;   // tensor-core kernels: set to 1 when a bounded wait gives up
     int64_t sf_cols;       // > 0: scale bytes in the block-scaled MMA layout, sf_cols = cols / B
     int64_t sf_kt;         //   ... with sf_kt = ceil(sf_cols / 4) 512-byte atoms per 128-row block
 };
@@ -536,9 +535,11 @@ __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, cons
 }
 
 // Scale, codes, MSE terms, dequantized values and stores of unit u, whose
-// (rotated) values are v and whose blocks' absolute maxima are m.
-template <int FMT, int B, int K, bool MSE, bool DQ>
-__device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u, const f32x2 (&v)[EPT / 2],
+// blocks' absolute maxima are m and whose (rotated) values are produced half
+// by half: half(h, vh) fills vh with elements 16 h .. 16 h + 15 as 8 pairs
+// (h = 0 then 1), so a caller can hold only half of the unit in registers.
+template <int FMT, int B, int K, bool MSE, bool DQ, typename Half>
+__device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u, Half&& half,
                                                 const float (&m)[UnitShape<B, K>::NB], int lane,
                                                 const ScaleConsts& kc, const float2* tab, float nz,
                                                 double (&acc)[3], uint64_t pol)
@@ -563,10 +564,12 @@ __device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u,
 #pragma unroll
         for (int bi = 0; bi < NB; ++bi) anyzero |= sc[bi] == 0.0f;
     }
+    f32x2 vh[EPT / 4];
 #pragma unroll
     for (int k = 0; k < EPT / 8; ++k) {
         const int bi = (8 * k) / BE;
-        const f32x2* vk = v + 4 * k;
+        if ((k & 1) == 0) half(k >> 1, vh);
+        const f32x2* vk = vh + 4 * (k & 1);
         uint32_t h[4];
         if constexpr (FMT == kE8M0) {
             // S is a power of two: y * (1/S) is the quotient itself.
@@ -675,6 +678,22 @@ __device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u,
 
     // ---- stores
     store_unit<B, K, DQ>(p, u, cw, code, lane, pol);
+}
+
+// The same for a unit held whole in registers.
+template <int FMT, int B, int K, bool MSE, bool DQ>
+__device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u, const f32x2 (&v)[EPT / 2],
+                                                const float (&m)[UnitShape<B, K>::NB], int lane,
+                                                const ScaleConsts& kc, const float2* tab, float nz,
+                                                double (&acc)[3], uint64_t pol)
+{
+    quantize_halves<FMT, B, K, MSE, DQ>(
+        p, u,
+        [&](int h, f32x2 (&vh)[EPT / 4]) {
+#pragma unroll
+            for (int j = 0; j < EPT / 4; ++j) vh[j] = v[(EPT / 4) * h + j];
+        },
+        m, lane, kc, tab, nz, acc, pol);
 }
 
 template <int FMT, int B, int K, bool MSE, bool DQ>
@@ -902,7 +921,6 @@ struct AmaxParams {
     int64_t n;
     unsigned int* amax_bits;   // max |y| as fp32 bits (non-negative floats order as integers)
     float c_hi, c_lo;
-    unsigned int* fault;       // tensor-core kernel: set to 1 when a bounded wait gives up
 };
 
 template <int K>

@@ -20,15 +20,6 @@ int resident_ctas(const void* kernel, int smem, int threads = 256);
 // the tensor cores gives up instead of hanging.
 unsigned int* device_fault_word();
 
-// A 2-D TMA tensor map (driver's cuTensorMapEncodeTiled, fetched once at run
-// time): inner dimension `inner` elements of `elem_bytes` bytes, `rows` rows
-// `row_bytes` apart, boxes of box_inner x box_rows, the given swizzle
-// (CUtensorMapSwizzle value), zero fill out of bounds.  `map` points to a
-// 64-byte aligned 128-byte CUtensorMap.  False if the encoder is unavailable
-// or rejects the arguments.
-bool encode_tensor_map_2d(void* map, int elem_bytes, const void* base, uint64_t inner, uint64_t rows,
-                          uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle);
-
 // Grid for a grid-stride kernel: min(ctas_needed, resident CTAs), at least 1.
 int grid_for(const void* kernel, int smem, int64_t ctas_needed, int threads = 256);
 

@@ -5,7 +5,6 @@
 
 #include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
-#include "fp4q_tc.cuh"
 
 namespace fp4q {
 
@@ -27,42 +26,6 @@ unsigned int* device_fault_word()
     return static_cast<unsigned int*>(p);
 }
 
-namespace {
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static std::once_flag once;
-    static EncodeTiledFn fn = nullptr;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    });
-    return fn;
-}
-}  // namespace
-
-bool encode_tensor_map_2d(void* map, int elem_bytes, const void* base, uint64_t inner, uint64_t rows,
-                          uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle)
-{
-    EncodeTiledFn enc = encode_fn();
-    if (!enc || rows == 0 || inner == 0) return false;
-    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(static_cast<CUtensorMap*>(map), dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, static_cast<CUtensorMapSwizzle>(swizzle),
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int resident_ctas(const void* kernel, int smem, int threads)
 {
     static std::mutex mu;
@@ -76,9 +39,33 @@ int resident_ctas(const void* kernel, int smem, int threads)
         if (it != cache.end()) return it->second;
     }
     if (smem > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // Prefer the largest shared-memory carveout: these kernels stage their input in
+    // shared memory and barely use L1, and without a preference the carveout may be
+    // sized for a single CTA, capping residency at one CTA per SM.
+    cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     int sms = 0, occ = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem);
+    // The same bound from the kernel's registers, shared memory and threads (the
+    // occupancy query reports one CTA per SM for kernels that use tensor memory;
+    // the hardware co-schedules more, up to these limits).
+    cudaFuncAttributes fa;
+    int smem_sm = 0, smem_rsv = 0, thr_sm = 0;
+    if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) == cudaSuccess) {
+        const int warps = (threads + 31) / 32;
+        const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
+        const int by_regs = regs_warp > 0 ? 65536 / (regs_warp * warps) : 32;
+        const int cta_smem = (int)fa.sharedSizeBytes + smem + smem_rsv;
+        const int by_smem = cta_smem > 0 ? smem_sm / cta_smem : 32;
+        const int by_thr = thr_sm / (warps * 32);
+        int manual = by_regs < by_smem ? by_regs : by_smem;
+        if (by_thr < manual) manual = by_thr;
+        if (manual > 32) manual = 32;
+        if (manual > occ) occ = manual;
+    }
     const int resident = (sms > 0 ? sms : 1) * (occ > 0 ? occ : 1);
     std::lock_guard<std::mutex> lock(mu);
     cache[key] = resident;
@@ -115,27 +102,6 @@ namespace {
 template <int K>
 cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
-    // the rotation on the tensor cores, 4096-element tiles through a TMA ring of
-    // 32-element rows; a tensor whose size is an odd multiple of 16 rotates with
-    // the butterfly kernel below
-    if constexpr (K == 16 || K == 32) {
-        if (p.n % 32 == 0) {
-            TcAmaxParams tp;
-            memset(&tp, 0, sizeof(tp));
-            tp.p = p;
-            tp.p.fault = device_fault_word();
-            if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
-            if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
-                                      tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
-                return cudaErrorInvalidValue;
-            auto kern = amax_tc_kernel<K>;
-            const int64_t tiles = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
-            const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, tiles, tc::THREADS);
-            if (pdl) return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
-            kern<<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(tp);
-            return cudaGetLastError();
-        }
-    }
     auto kern = amax_kernel<K>;
     const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));
     if (pdl) return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);

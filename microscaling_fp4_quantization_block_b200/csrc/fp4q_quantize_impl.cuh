@@ -6,7 +6,6 @@
 
 #include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
-#include "fp4q_tc.cuh"
 
 namespace fp4q {
 namespace detail {
@@ -14,27 +13,6 @@ namespace detail {
 template <int FMT, int B, int K, bool MSE, bool DQ = false>
 cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
 {
-    // the rotation on the tensor cores, 4096-element tiles through a TMA ring of
-    // 32-element rows; a tensor whose size is an odd multiple of 16 (cols = 16
-    // mod 32, K = 16) rotates with the butterfly kernel below
-    if constexpr (K == 16 || K == 32) {
-        if (p.n % 32 == 0) {
-            TcQuantParams tp;
-            memset(&tp, 0, sizeof(tp));
-            tp.p = p;
-            tp.p.fault = device_fault_word();
-            if (tp.p.fault == nullptr) return cudaErrorInvalidDevice;
-            if (!encode_tensor_map_2d(&tp.xmap, 2, p.x, tc::KR, (uint64_t)(p.n / tc::KR), 2 * tc::KR, tc::KR,
-                                      tc::ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
-                return cudaErrorInvalidValue;
-            auto kern = quantize_tc_kernel<FMT, B, K, MSE, DQ>;
-            int64_t need = (p.n + tc::TILE_ELEMS - 1) / tc::TILE_ELEMS;
-            if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
-            const int grid = grid_for((const void*)kern, tc::SMEM_BYTES, need, tc::THREADS);
-            if (grid_out) *grid_out = grid;
-            return launch_pdl(kern, grid, tc::THREADS, tc::SMEM_BYTES, s, tp);
-        }
-    }
     auto kern = quantize_kernel<FMT, B, K, MSE, DQ>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);

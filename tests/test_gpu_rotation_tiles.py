@@ -1,13 +1,10 @@
-"""The Hadamard rotation on the tensor cores (rotations of 16 and 32, "Bridging
-the Gap", s3.1: block-wise rotation fused with quantization), through the C ABI.
-
-The quantize kernels with rot 16 / 32 rotate with tcgen05.mma (bf16 operands,
-fp32 accumulators in tensor memory) instead of fp32 butterflies; the results
-obey the same rotated-path rule against the oracle's fp64 rotation.  These
-cases walk the warpgroup pipeline through its edges: one partial tile, exactly
-one and two tiles, several tiles per warpgroup (both accumulator buffers and
-both mbarrier phases reused many times), and every scale format, with the
-device fault word checked after each run.
+"""Rotations of 16 and 32 ("Bridging the Gap", s3.1: block-wise rotation fused
+with quantization), through the C ABI, at the edges of the kernels' work
+decomposition: one partial tile, exactly one and two 1024-element tiles, many
+tiles per warp (the shared-memory ring wrapping round many times), and every
+scale format; the fused kernel's codes, scales, dequantized values and MSE, and
+the rotated maximum.  The results obey the rotated-path rule against the
+oracle's fp64 rotation; the device fault word stays 0.
 """
 import numpy as np
 import pytest
@@ -36,8 +33,8 @@ def fq():
 @pytest.mark.parametrize("rows,cols", [(1, 32), (3, 1024), (4, 1024), (8, 1024), (7, 4096), (300, 2048)])
 @pytest.mark.parametrize("rot", [16, 32])
 def test_tile_edges(fq, rows, cols, rot):
-    """n = 32 (one row of one partial tile), 3072, 4096 (one tile), 8192 (two),
-    28672 and 614400 elements."""
+    """n = 32 (one row of one partial tile), 3072, 4096, 8192, 28672 and
+    614400 elements."""
     x, _ = workloads.student_t_outliers_bf16(rows, cols, seed=rows * cols + rot, n_outlier=min(8, cols))
     xb = bf16_bits(x)
     for fmt, block, gmode in [(E8, 32, NONE), (U4, 16, COMP), (U4, 8, NONE), (U5, 32, NONE)]:
@@ -49,7 +46,7 @@ def test_tile_edges(fq, rows, cols, rot):
 
 @pytest.mark.parametrize("rot", [16, 32])
 def test_many_tiles_per_warpgroup_fused(fq, rot):
-    """2048 x 5120 elements: 2560 tiles, several per warpgroup; the fused
+    """2048 x 5120 elements: 10240 tiles of 1024, several per warp; the fused
     kernel's codes, scales, dequantized values and MSE against the oracle."""
     x, _ = workloads.student_t_outliers_bf16(2048, 5120, seed=11 + rot)
     xd = x.cuda()
@@ -73,8 +70,8 @@ def test_many_tiles_per_warpgroup_fused(fq, rot):
 
 @pytest.mark.parametrize("rot", [16, 32])
 def test_rotated_amax(fq, rot):
-    """max |y| over the tensor-core rotation against the exact rotation: equal up
-    to the rotation's rounding."""
+    """max |y| of the rotated tensor against the exact rotation: equal up to the
+    rotation's rounding."""
     x, _ = workloads.student_t_outliers_bf16(1000, 2048, seed=rot)
     amax = fq.fp4q_tensor_amax(x.cuda(), rot)
     torch.cuda.synchronize()
