@@ -52,9 +52,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;   // 36 KiB
 constexpr int SMEM_BYTES = 1024 + NSTAGE * STAGE_BYTES + 256;
 constexpr int EPI_WARPS = 4;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
-constexpr uint32_t TMEM_COLS = 512;         // two 128-column accumulators + the scale ring, 4 x 32
+constexpr uint32_t TMEM_COLS = 512;         // two 128-column accumulators + the scale ring, NSTAGE x 32
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 2 * BN;
+static_assert(SF_COL + NSTAGE * 32 <= TMEM_COLS, "tensor memory: accumulators and scale ring");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 constexpr uint32_t kMaxPolls = 1u << 24;
 
 struct Params {

@@ -948,13 +948,21 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
                              asm("max.u16x2 %0, %0, %1;" : "+r"(mb) : "r"(a));
                          }
                      } else {
+                         // the raw Sylvester sums; 1/sqrt(K) is applied once, to the maximum
                          f32x2 v[EPT / 2];
                          unpack_unit(w, v);
-                         rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+                         fwht_inreg<EPT, (K < EPT ? K : EPT)>(v);
+                         if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(v, lane);
                          mx = fmaxf(mx, pairs_absmax<EPT>(v));
                      }
                  });
-    if constexpr (K == 0) mx = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
+    if constexpr (K == 0) {
+        mx = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
+    } else {
+        // y = fp32(s c_hi + fp32(s c_lo)) rounds monotonically and symmetrically in s, so
+        // the largest |y| is the normalised largest |s|: the quantizer's own maxima exactly
+        mx = __fmaf_rn(mx, p.c_hi, __fmul_rn(mx, p.c_lo));
+    }
     mx = group_max<32>(mx);
     if (lane == 0 && mx > 0.0f) atomicMax(p.amax_bits, __float_as_uint(mx));
 }
