@@ -153,6 +153,21 @@ FP4Q_API int fp4q_tensor_amax_accumulate(const void* x, int64_t rows, int64_t co
                                          void* stream);
 
 /*
+ * fp4q_tensor_amax_batched -- the maxima of `count` tensors in one pass:
+ * *amax[i] = max |y| over tensor i (accumulate = 0), or max(*amax[i], that)
+ * (accumulate != 0, as fp4q_tensor_amax_accumulate).  All tensors take the
+ * same rot.  The host arrays xs, rows, cols and amax (count entries each) are
+ * read during the call only; the tensors' tiles are laid end to end and
+ * streamed by one kernel launch per 32 tensors, so many small tensors (the
+ * projections of a model layer) cost about what one tensor of their total
+ * size does.  Slots must be distinct within a call.  Every tensor is checked
+ * before anything is enqueued; errors as for fp4q_tensor_amax, and
+ * FP4Q_ERR_SHAPE for count < 0 (count = 0 does nothing).
+ */
+FP4Q_API int fp4q_tensor_amax_batched(int count, const void* const* xs, const int64_t* rows, const int64_t* cols,
+                                      int rot, float* const* amax, int accumulate, void* stream);
+
+/*
  * fp4q_global_scale -- *gscale = amax / (6 * 448) (correctly rounded fp32), or
  * 1 when amax = 0: the per-tensor scale of COMPUTE mode from an absolute
  * maximum that is already known (for instance one reduced across several

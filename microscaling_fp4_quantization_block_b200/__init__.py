@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
         "fp4q_outlier_stats_workspace_size": (SZ, []),
         "fp4q_tensor_amax": (I, [P, I64, I64, I, P, P]),
         "fp4q_tensor_amax_accumulate": (I, [P, I64, I64, I, P, P]),
+        "fp4q_tensor_amax_batched": (I, [I, P, P, P, I, P, I, P]),
         "fp4q_global_scale": (I, [P, P, P]),
         "fp4q_dequantize": (I, [P, P, P, I64, I64, I, I, I, I, P, P]),
         "fp4q_block_mse": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P, SZ, P]),
@@ -311,6 +312,32 @@ def fp4q_tensor_amax_accumulate(x: torch.Tensor, amax: torch.Tensor, rot: int = 
     x = x.contiguous()
     st = lib().fp4q_tensor_amax_accumulate(_ptr(x), x.shape[0], x.shape[1], rot, _ptr(amax), _stream(stream))
     _check(st, "fp4q_tensor_amax_accumulate")
+    return amax
+
+
+def fp4q_tensor_amax_batched(xs, rot: int = 0, amax: Optional[torch.Tensor] = None, accumulate: bool = False,
+                             stream=None) -> torch.Tensor:
+    """max |y| of every tensor of xs (2-D bf16 CUDA tensors) in one pass:
+    amax[i] (a float32 CUDA tensor of len(xs) entries, allocated if None) is
+    set to, or with accumulate raised to, tensor i's maximum."""
+    xs = list(xs)
+    for x in xs:
+        if x.dtype != torch.bfloat16 or x.dim() != 2:
+            raise ValueError("every x must be a 2-D bf16 tensor")
+    _need_cuda(*xs)
+    xs = [x.contiguous() for x in xs]
+    if amax is None:
+        amax = torch.zeros((len(xs),), dtype=torch.float32, device=xs[0].device if xs else "cuda")
+    if amax.dtype != torch.float32 or amax.numel() < len(xs):
+        raise ValueError("amax must be a float32 tensor of len(xs) entries")
+    _need_cuda(amax)
+    n = len(xs)
+    ptrs = (ctypes.c_void_p * max(n, 1))(*[_ptr(x) for x in xs])
+    rows = (ctypes.c_int64 * max(n, 1))(*[x.shape[0] for x in xs])
+    cols = (ctypes.c_int64 * max(n, 1))(*[x.shape[1] for x in xs])
+    slots = (ctypes.c_void_p * max(n, 1))(*[amax.data_ptr() + 4 * i for i in range(n)])
+    st = lib().fp4q_tensor_amax_batched(n, ptrs, rows, cols, rot, slots, 1 if accumulate else 0, _stream(stream))
+    _check(st, "fp4q_tensor_amax_batched")
     return amax
 
 

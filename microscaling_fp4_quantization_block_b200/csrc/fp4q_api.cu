@@ -84,9 +84,12 @@ cudaError_t enqueue_amax(const void* x, int64_t n, int rot, float* dst, cudaStre
     }
     if (n == 0) return cudaSuccess;
     AmaxParams ap{};
-    ap.x = static_cast<const uint16_t*>(x);
-    ap.n = n;
-    ap.amax_bits = reinterpret_cast<unsigned int*>(dst);
+    ap.count = 1;
+    ap.x[0] = static_cast<const uint16_t*>(x);
+    ap.n[0] = n;
+    ap.tile0[0] = 0;
+    ap.tile0[1] = (n + kAmaxTileElems - 1) / kAmaxTileElems;
+    ap.amax_bits[0] = reinterpret_cast<unsigned int*>(dst);
     rotation_constants(rot, &ap.c_hi, &ap.c_lo);
     return launch_amax(rot, ap, s, !zero);
 }
@@ -356,6 +359,39 @@ int fp4q_tensor_amax_accumulate(const void* x, int64_t rows, int64_t cols, int r
     if (!amax || (n > 0 && !x)) return FP4Q_ERR_NULL;
     if (!aligned(amax, 4) || (n > 0 && !aligned(x, 32))) return FP4Q_ERR_ALIGN;
     return cuda_status(enqueue_amax(x, n, rot, amax, as_stream(stream), false));
+}
+
+int fp4q_tensor_amax_batched(int count, const void* const* xs, const int64_t* rows, const int64_t* cols, int rot,
+                             float* const* amax, int accumulate, void* stream)
+{
+    if (count < 0) return FP4Q_ERR_SHAPE;
+    if (count == 0) return FP4Q_OK;
+    if (!xs || !rows || !cols || !amax) return FP4Q_ERR_NULL;
+    for (int i = 0; i < count; ++i) {                 // every tensor checked before anything is enqueued
+        int64_t n = 0;
+        int st = check_shape(rows[i], cols[i], FP4Q_SCALE_E8M0, 8, rot, &n);
+        if (st) return st;
+        if (!amax[i] || (n > 0 && !xs[i])) return FP4Q_ERR_NULL;
+        if (!aligned(amax[i], 4) || (n > 0 && !aligned(xs[i], 32))) return FP4Q_ERR_ALIGN;
+    }
+    cudaStream_t s = as_stream(stream);
+    for (int c0 = 0; c0 < count; c0 += kAmaxBatch) {
+        AmaxParams ap{};
+        ap.count = count - c0 < kAmaxBatch ? count - c0 : kAmaxBatch;
+        rotation_constants(rot, &ap.c_hi, &ap.c_lo);
+        ap.tile0[0] = 0;
+        for (int j = 0; j < ap.count; ++j) {
+            ap.x[j] = static_cast<const uint16_t*>(xs[c0 + j]);
+            ap.n[j] = rows[c0 + j] * cols[c0 + j];
+            ap.tile0[j + 1] = ap.tile0[j] + (ap.n[j] + kAmaxTileElems - 1) / kAmaxTileElems;
+            ap.amax_bits[j] = reinterpret_cast<unsigned int*>(amax[c0 + j]);
+        }
+        cudaError_t e = cudaSuccess;
+        if (!accumulate) e = launch_amax_zero(ap, s);
+        if (e == cudaSuccess && ap.tile0[ap.count] > 0) e = launch_amax(rot, ap, s, true);
+        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    return FP4Q_OK;
 }
 
 int fp4q_global_scale(const float* amax, float* gscale, void* stream)

@@ -441,11 +441,12 @@ __device__ __forceinline__ ScaleConsts scale_consts(float G)
 // Values are held as N/2 fp32 pairs p[k] = (v[2k], v[2k+1]).  In-register
 // Sylvester Hadamard transform of every run of CH consecutive values (natural
 // order: y_i = sum_j (-1)^popcount(i & j) x_j): the distance-1 stage mixes the
-// two halves of each pair, the others combine whole pairs.
-template <int N, int CH>
+// two halves of each pair, the others combine whole pairs.  FIRST = false
+// skips the distance-1 stage (done already by unpack_fwht2).
+template <int N, int CH, bool FIRST = true>
 __device__ __forceinline__ void fwht_inreg(f32x2 (&p)[N / 2])
 {
-    if constexpr (CH >= 2) {
+    if constexpr (FIRST && CH >= 2) {
 #pragma unroll
         for (int k = 0; k < N / 2; ++k) {
             float a, b;
@@ -463,6 +464,31 @@ __device__ __forceinline__ void fwht_inreg(f32x2 (&p)[N / 2])
                 p[(i + h) / 2] = sub2(a, b);
             }
         }
+    }
+}
+
+// bf16 words -> fp32 pairs with the distance-1 butterfly stage folded in:
+// p[k] = (x0 + x1, x1 - x0) for w[k] = (x0, x1), each a single rounding of the
+// exact sum or difference (mixed-precision add / subtract of the bf16 high
+// half and the widened low half), so three instructions per pair instead of
+// the widening (two) plus the stage (two).  The second value of every pair is
+// the NEGATED distance-1 difference.  Every later stage, in registers or
+// across lanes, combines like positions linearly, so the odd positions stay
+// negated to the end of the transform, where the normalisation multiplies
+// them by -c (RN(-a) = -RN(a): the values are exactly those of the plain
+// transform).
+template <int N>
+__device__ __forceinline__ void unpack_fwht2(const uint32_t (&w)[N / 2], f32x2 (&p)[N / 2])
+{
+#pragma unroll
+    for (int k = 0; k < N / 2; ++k) {
+        const float lo = bf16_lo(w[k]);
+        float s, d;
+        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tadd.rn.f32.bf16 %0, h, %3;\n\t"
+            "sub.rn.f32.bf16 %1, h, %3;\n\t}"
+            : "=f"(s), "=f"(d)
+            : "r"(w[k]), "f"(lo));
+        p[k] = pk(s, d);
     }
 }
 

@@ -129,8 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) gscale_search_kernel(GscaleParams
                      uint32_t w[EPT / 2];
                      ring.read(s, 0, w);
                      f32x2 v[EPT / 2];
-                     unpack_unit(w, v);
-                     rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+                     load_unit<K>(w, v, lane, p.c_hi, p.c_lo);
                      float m[S::NB];
                      if constexpr (K == 0) block_max_words<B>(w, m);
                      else block_max<B, K>(v, m);

@@ -139,31 +139,25 @@ __device__ __forceinline__ R warp_ring(uint8_t* smem)
 }
 
 // Ring pipeline driver: calls body(tile, stage) for every tile of this warp,
-// with the tile's input resident in the ring.  NSTAGE - 1 tiles are in flight.
-// EF: the copies allocate their L2 lines evict-first (policy pol).
-template <bool EF = false, typename R, typename Body>
-__device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __restrict__ src, int64_t nbytes,
-                                             int64_t n_tiles, int64_t warp, int64_t n_warps, int lane,
-                                             Body&& body, uint64_t pol = 0)
+// with the tile's input resident in the ring; issue(tile, stage) starts the
+// copies of a tile.  NSTAGE - 1 tiles are in flight.
+template <int NS, typename Issue, typename Body>
+__device__ __forceinline__ void stream_tiles_with(int64_t n_tiles, int64_t warp, int64_t n_warps, Issue&& issue,
+                                                  Body&& body)
 {
-    constexpr int NS = R::NSTAGE;
-    const int64_t step = n_warps * R::TILE_BYTES;
     int64_t t_issue = warp;
-    int64_t off_issue = warp * R::TILE_BYTES;
 #pragma unroll
     for (int s = 0; s < NS - 1; ++s) {
-        if (t_issue < n_tiles) ring.template issue<EF>(src, nbytes, off_issue, s, lane, pol);
+        if (t_issue < n_tiles) issue(t_issue, s);
         cp_async_commit();
         t_issue += n_warps;
-        off_issue += step;
     }
     int stage = 0;
     for (int64_t t = warp; t < n_tiles; t += n_warps) {
         const int s_new = stage == 0 ? NS - 1 : stage - 1;          // the slot read last iteration
-        if (t_issue < n_tiles) ring.template issue<EF>(src, nbytes, off_issue, s_new, lane, pol);
+        if (t_issue < n_tiles) issue(t_issue, s_new);
         cp_async_commit();
         t_issue += n_warps;
-        off_issue += step;
         cp_async_wait<NS - 1>();                                   // tile t has landed (own copies)
         __syncwarp();                                              // ... and every lane's copies
         body(t, stage);
@@ -171,6 +165,18 @@ __device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __res
         __syncwarp();                                              // slot may be refilled next iteration
     }
     cp_async_wait_all();
+}
+
+// The same over one contiguous input of nbytes bytes, tile t at byte t * TILE_BYTES.
+// EF: the copies allocate their L2 lines evict-first (policy pol).
+template <bool EF = false, typename R, typename Body>
+__device__ __forceinline__ void stream_tiles(const R& ring, const uint8_t* __restrict__ src, int64_t nbytes,
+                                             int64_t n_tiles, int64_t warp, int64_t n_warps, int lane,
+                                             Body&& body, uint64_t pol = 0)
+{
+    stream_tiles_with<R::NSTAGE>(
+        n_tiles, warp, n_warps,
+        [&](int64_t t, int s) { ring.template issue<EF>(src, nbytes, t * R::TILE_BYTES, s, lane, pol); }, body);
 }
 
 using XRing = Ring<2 * EPT, 1>;                                  // one bf16 unit per lane per tile
@@ -183,15 +189,55 @@ __device__ __forceinline__ void unpack_unit(const uint32_t (&w)[EPT / 2], f32x2 
     for (int k = 0; k < EPT / 2; ++k) p[k] = pk(bf16_lo(w[k]), bf16_hi_fp(w[k]));
 }
 
-// Optional rotation of a unit held in registers: runs of K elements, the part
-// inside the unit in registers, the rest across lanes, then 1/sqrt(K).
+// The Sylvester sums of a unit's runs of K elements (K > 0): the part of a run
+// inside the unit in registers, the rest across lanes.  The odd positions come
+// out negated (see unpack_fwht2); only magnitudes are read from the result, or
+// normalise_signed restores the signs.
 template <int K>
-__device__ __forceinline__ void rotate_unit(f32x2 (&p)[EPT / 2], int lane, float c_hi, float c_lo)
+__device__ __forceinline__ void unit_sums(const uint32_t (&w)[EPT / 2], f32x2 (&p)[EPT / 2], int lane)
 {
-    if constexpr (K > 0) {
-        fwht_inreg<EPT, (K < EPT ? K : EPT)>(p);
-        if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(p, lane);
-        normalize<EPT>(p, c_hi, c_lo);
+    static_assert(K >= 2, "rotation runs of at least two elements");
+    unpack_fwht2<EPT>(w, p);
+    fwht_inreg<EPT, (K < EPT ? K : EPT), false>(p);
+    if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(p, lane);
+}
+
+// y = s / sqrt(K) rounded to fp32, the odd positions' signs restored by
+// multiplying them by the negated constant.  K = 16: 1/sqrt(K) = 1/4 is exact,
+// one product per value.  K = 32, 128: the constant is split as c_hi + c_lo
+// (both fp32, from the fp64 value) and y = fp32(s c_hi + fp32(s c_lo)), the
+// fp32 value nearest to s / sqrt(K) except within ~2^-47 (relative) of a
+// rounding midpoint (a single product by c_hi would add up to 0.14 ulp, and
+// with it codes that differ from the exact rotation's at E2M1 ties).  Every
+// rounding adds +0 last, which leaves non-zero values as they are and makes
+// every zero +0: an exact cancellation in a negated position would otherwise
+// come out as -0, while a zero of the exact rotation (a sum that starts from
+// +0) is +0.
+template <int K>
+__device__ __forceinline__ void normalise_signed(f32x2 (&p)[EPT / 2], float c_hi, float c_lo)
+{
+    const f32x2 hi = pk(c_hi, -c_hi), z = pk(0.0f, 0.0f);
+    if constexpr (K == 16) {
+#pragma unroll
+        for (int k = 0; k < EPT / 2; ++k) p[k] = fma2(p[k], hi, z);
+    } else {
+        const f32x2 lo = pk(c_lo, -c_lo);
+#pragma unroll
+        for (int k = 0; k < EPT / 2; ++k) p[k] = fma2(p[k], hi, fma2(p[k], lo, z));
+    }
+}
+
+// A unit's values for quantization: the widened bf16 inputs (K = 0), or their
+// rotation by H_K / sqrt(K) over runs of K elements.
+template <int K>
+__device__ __forceinline__ void load_unit(const uint32_t (&w)[EPT / 2], f32x2 (&p)[EPT / 2], int lane, float c_hi,
+                                          float c_lo)
+{
+    if constexpr (K == 0) {
+        unpack_unit(w, p);
+    } else {
+        unit_sums<K>(w, p, lane);
+        normalise_signed<K>(p, c_hi, c_lo);
     }
 }
 
@@ -703,8 +749,7 @@ __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, c
 {
     using S = UnitShape<B, K>;
     f32x2 v[EPT / 2];
-    unpack_unit(w, v);
-    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+    load_unit<K>(w, v, lane, p.c_hi, p.c_lo);
     float m[S::NB];
     if constexpr (K == 0) block_max_words<B>(w, m);
     else block_max<B, K>(v, m);
@@ -797,8 +842,7 @@ __device__ __forceinline__ void search_unit(const QuantParams& p, int64_t u, con
     using S = UnitShape<B, K>;
     constexpr int NB = S::NB, BE = S::BE;
     f32x2 v[EPT / 2];
-    unpack_unit(w, v);
-    rotate_unit<K>(v, lane, p.c_hi, p.c_lo);
+    load_unit<K>(w, v, lane, p.c_hi, p.c_lo);
     float m[NB];
     if constexpr (K == 0) block_max_words<B>(w, m);
     else block_max<B, K>(v, m);
@@ -916,11 +960,20 @@ __global__ void __launch_bounds__(kThreads, 2) search_kernel(QuantParams p)
 }
 
 // ---------------------------------------------------------------- per-tensor amax
+// One launch takes the maxima of up to kAmaxBatch tensors: their ring tiles are
+// numbered one after the other (tensor c owns tiles tile0[c] .. tile0[c+1]-1),
+// and the warps stride over all of them, so a batch of small tensors fills the
+// GPU like one large tensor.
+constexpr int kAmaxBatch = 32;
+constexpr int kAmaxTileElems = 32 * EPT;    // elements of one ring tile
+
 struct AmaxParams {
-    const uint16_t* x;
-    int64_t n;
-    unsigned int* amax_bits;   // max |y| as fp32 bits (non-negative floats order as integers)
-    float c_hi, c_lo;
+    const uint16_t* x[kAmaxBatch];
+    int64_t n[kAmaxBatch];                  // elements of each tensor
+    int64_t tile0[kAmaxBatch + 1];          // first tile of each tensor; tile0[count] = all tiles
+    unsigned int* amax_bits[kAmaxBatch];    // max |y| as fp32 bits (non-negative floats order as integers)
+    int count;
+    float c_hi, c_lo;                       // 1/sqrt(K) split in two fp32 parts
 };
 
 template <int K>
@@ -930,41 +983,68 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
     pdl_release();
     extern __shared__ __align__(128) uint8_t smem_ring[];
     const int lane = threadIdx.x & 31;
-    const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
+    const int64_t n_tiles = p.tile0[p.count];
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
     const XRing ring = warp_ring<XRing>(smem_ring);
+    // A warp's tiles rise, so its tensors do too: one cursor for the copies issued
+    // ahead and one for the tile being reduced.  Tiles past tile0[count] are never
+    // issued, so both cursors stay below count.
+    int ci = 0, cb = 0, cur = -1;
     float mx = 0.0f;
     uint32_t mb = 0;                                       // max |bf16| pattern, two halves
-    stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
-                 [&](int64_t, int s) {
-                     uint32_t w[EPT / 2];
-                     ring.read(s, 0, w);
-                     if constexpr (K == 0) {
-                         // |bf16| patterns order like their values: SIMD max of both halves
+    auto flush = [&]() {
+        float m;
+        if constexpr (K == 0) {
+            m = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
+        } else {
+            // y = fp32(s c_hi + fp32(s c_lo)) rounds monotonically and symmetrically in s
+            // (c_lo = 0 for K = 16), so the largest |y| is the normalised largest |s|: the
+            // quantizer's own maxima exactly
+            m = __fmaf_rn(mx, p.c_hi, __fmul_rn(mx, p.c_lo));
+        }
+        m = group_max<32>(m);
+        if (lane == 0 && m > 0.0f) atomicMax(p.amax_bits[cur], __float_as_uint(m));
+        mx = 0.0f;
+        mb = 0;
+    };
+    stream_tiles_with<XRing::NSTAGE>(
+        n_tiles, warp, n_warps,
+        [&](int64_t t, int s) {
+            while (t >= p.tile0[ci + 1]) ++ci;
+            ring.issue(reinterpret_cast<const uint8_t*>(p.x[ci]), 2 * p.n[ci], (t - p.tile0[ci]) * XRing::TILE_BYTES,
+                       s, lane);
+        },
+        [&](int64_t t, int s) {
+            while (t >= p.tile0[cb + 1]) ++cb;
+            if (cb != cur) {                                // warp-uniform: the tile is the warp's
+                if (cur >= 0) flush();
+                cur = cb;
+            }
+            uint32_t w[EPT / 2];
+            ring.read(s, 0, w);
+            if constexpr (K == 0) {
+                // |bf16| patterns order like their values: SIMD max of both halves
 #pragma unroll
-                         for (int k = 0; k < EPT / 2; ++k) {
-                             const uint32_t a = w[k] & 0x7fff7fffu;
-                             asm("max.u16x2 %0, %0, %1;" : "+r"(mb) : "r"(a));
-                         }
-                     } else {
-                         // the raw Sylvester sums; 1/sqrt(K) is applied once, to the maximum
-                         f32x2 v[EPT / 2];
-                         unpack_unit(w, v);
-                         fwht_inreg<EPT, (K < EPT ? K : EPT)>(v);
-                         if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(v, lane);
-                         mx = fmaxf(mx, pairs_absmax<EPT>(v));
-                     }
-                 });
-    if constexpr (K == 0) {
-        mx = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
-    } else {
-        // y = fp32(s c_hi + fp32(s c_lo)) rounds monotonically and symmetrically in s, so
-        // the largest |y| is the normalised largest |s|: the quantizer's own maxima exactly
-        mx = __fmaf_rn(mx, p.c_hi, __fmul_rn(mx, p.c_lo));
-    }
-    mx = group_max<32>(mx);
-    if (lane == 0 && mx > 0.0f) atomicMax(p.amax_bits, __float_as_uint(mx));
+                for (int k = 0; k < EPT / 2; ++k) {
+                    const uint32_t a = w[k] & 0x7fff7fffu;
+                    asm("max.u16x2 %0, %0, %1;" : "+r"(mb) : "r"(a));
+                }
+            } else {
+                // the raw Sylvester sums (magnitudes only: their signs do not
+                // matter); 1/sqrt(K) is applied once, to the maximum
+                f32x2 v[EPT / 2];
+                unit_sums<K>(w, v, lane);
+                mx = fmaxf(mx, pairs_absmax<EPT>(v));
+            }
+        });
+    if (cur >= 0) flush();
+}
+
+// Zero the amax slots of a batch (before a batch that overwrites them).
+static __global__ void amax_zero_kernel(AmaxParams p)
+{
+    if ((int)threadIdx.x < p.count) *p.amax_bits[threadIdx.x] = 0u;
 }
 
 // G = amax / (6 * 448) (correctly rounded), or 1 for an all-zero tensor.
@@ -1394,8 +1474,7 @@ __global__ void __launch_bounds__(kThreads) block_mse_kernel(MseParams p)
         ring.read(s, 0, w);
         const int64_t e0 = u * EPT;
         f32x2 yp[EPT / 2];
-        unpack_unit(w, yp);
-        rotate_unit<K>(yp, lane, p.c_hi, p.c_lo);
+        load_unit<K>(w, yp, lane, p.c_hi, p.c_lo);
         float m[NB];
         block_max<B, K>(yp, m);
         float y[EPT], v[EPT];

@@ -39,6 +39,7 @@ cudaError_t launch_quantize_ue5m3(int B, int K, bool mse, const QuantParams& p, 
 // Quantize with MSE-optimised block scales (p.below / p.above candidate codes).
 cudaError_t launch_quantize_search(int fmt, int B, int K, const QuantParams& p, cudaStream_t s);
 cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl);
+cudaError_t launch_amax_zero(const AmaxParams& p, cudaStream_t s);
 // Outlier statistics: zeroes the histogram (workspace), stats and col_absmax,
 // then one histogram pass over x and a one-CTA scan.
 cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, double p, float* stats,

@@ -103,13 +103,20 @@ template <int K>
 cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
     auto kern = amax_kernel<K>;
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));
+    const int64_t tiles = p.tile0[p.count];
+    const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
     if (pdl) return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
     kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_amax_zero(const AmaxParams& p, cudaStream_t s)
+{
+    amax_zero_kernel<<<1, kAmaxBatch, 0, s>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_amax(int K, const AmaxParams& p, cudaStream_t s, bool pdl)
 {

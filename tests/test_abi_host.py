@@ -198,3 +198,31 @@ def test_global_scale_search_rejects_bad_arguments(fp4q):
     assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32 + 2, None, A32, ws, None) == -3
     assert g(A32, 4, 64, 1, 16, 0, 1, 1, A32, A32 + 4, A32, ws, None) == -3
     assert g(A32 + 16, 4, 64, 1, 16, 0, 1, 1, A32, None, A32, ws, None) == -3
+
+
+def test_batched_amax_rejects_bad_arguments(fp4q):
+    L = fp4q.lib()
+    f = L.fp4q_tensor_amax_batched
+
+    def arrs(xs, rows, cols, slots):
+        n = len(xs)
+        return ((ctypes.c_void_p * n)(*xs), (ctypes.c_int64 * n)(*rows), (ctypes.c_int64 * n)(*cols),
+                (ctypes.c_void_p * n)(*slots))
+
+    x, r, c, s = arrs([A32, A32], [4, 8], [64, 128], [A32, A32 + 4])
+    assert f(-1, x, r, c, 0, s, 0, None) == -2
+    assert f(0, None, None, None, 0, None, 0, None) == 0                          # nothing to do
+    assert f(2, None, r, c, 0, s, 0, None) == -1
+    assert f(2, x, r, c, 0, None, 0, None) == -1
+    assert f(2, x, r, c, 12, s, 0, None) == -4                                     # rot 12
+    assert f(2, *arrs([A32, A32], [4, 8], [64, 60], [A32, A32 + 4])[:3], 0, s, 0, None) == -2
+    assert f(2, *arrs([A32, A32], [4, -8], [64, 64], [A32, A32 + 4])[:3], 0, s, 0, None) == -2
+    assert f(2, *arrs([A32, A32], [4, 8], [64, 64], [A32, A32 + 4])[:3], 128, s, 0, None) == -2  # 64 % 128
+    xs, rs, cs, ss = arrs([A32, A32 + 16], [4, 8], [64, 128], [A32, A32 + 4])
+    assert f(2, xs, rs, cs, 0, ss, 0, None) == -3                                  # x not 32-byte aligned
+    xs, rs, cs, ss = arrs([A32, A32], [4, 8], [64, 128], [A32, A32 + 2])
+    assert f(2, xs, rs, cs, 0, ss, 0, None) == -3                                  # slot not 4-byte aligned
+    xs, rs, cs, ss = arrs([A32, None], [4, 8], [64, 128], [A32, A32 + 4])
+    assert f(2, xs, rs, cs, 0, ss, 0, None) == -1                                  # non-empty tensor, no data
+    xs, rs, cs, ss = arrs([A32, A32], [4, 8], [64, 128], [A32, None])
+    assert f(2, xs, rs, cs, 0, ss, 1, None) == -1

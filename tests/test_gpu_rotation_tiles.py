@@ -80,3 +80,32 @@ def test_rotated_amax(fq, rot):
     l1 = np.abs(xf.astype(np.float64)).reshape(-1, rot).sum(1).max() / np.sqrt(rot)
     assert abs(float(amax.item()) - want) <= (np.log2(rot) + 2) * 2.0 ** -24 * l1 + 2.0 ** -23 * want
     assert fq.fp4q_device_fault() == 0
+
+
+@pytest.mark.parametrize("rot", [16, 32, 128])
+def test_exact_cancellations_give_positive_zero(fq, rot):
+    """Runs whose rotated values cancel exactly: the oracle's rotation sums from
+    +0, so every zero rotated value is +0 and takes nibble 0x0, never the
+    negative-zero nibble 0x8.  Rows of pairwise-equal values make every odd
+    position of a run 0, rows of a value and its negation every even one, and
+    an all-zero row and one of -0 give 0 everywhere; the codes (and the scales)
+    are bit-exact there."""
+    rows, cols = 64, 1024
+    x, _ = workloads.student_t_outliers_bf16(rows, cols, seed=900 + rot, n_outlier=0)
+    x = x.float()
+    x[0::4, 1::2] = x[0::4, 0::2]                       # x1 = x0: odd Sylvester sums cancel
+    x[1::4, 1::2] = -x[1::4, 0::2]                      # x1 = -x0: even sums cancel
+    x[2] = 0.0
+    x[3] = -0.0
+    x = x.to(torch.bfloat16)
+    xb = bf16_bits(x)
+    for fmt, block, gmode in [(E8, 32, NONE), (U4, 16, COMP)]:
+        g = gpu_run(fq, x, fmt, block, rot, gmode, want_deq=False)
+        o = oracle_run(xb, fmt, block, rot, gmode, want_mse=False, want_deq=False)
+        gn = oracle.unpack_nibbles(g["codes"]).reshape(rows, cols)
+        on = oracle.unpack_nibbles(o["codes"]).reshape(rows, cols)
+        y, _ = __import__("_helpers").exact_rotation(oracle.bf16_bits_to_f32(xb), rot)
+        zero = y == 0.0
+        assert zero.sum() >= rows * cols // 4
+        assert (on[zero] == 0).all() and (gn[zero] == 0).all()
+        check_rotated(g, o, oracle.bf16_bits_to_f32(xb), fmt, block, rot)
