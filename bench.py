@@ -17,7 +17,8 @@ FP32 per-tensor scale), each without and with the 32-wide Hadamard rotation
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp4q|reference]
                     [--workload NAME]
 
-Prints one JSON line (rank 0).  Under torchrun each rank processes its own
+The timed steps replay the step's C-ABI calls as one CUDA graph, captured
+once (--no-graph: enqueue them call by call).  Prints one JSON line (rank 0).  Under torchrun each rank processes its own
 copy of the workload (independent tensors, no data-path collective): weak
 scaling, timed as the max over ranks of the device time.
 """
@@ -38,6 +39,7 @@ if ROOT not in sys.path:
 
 METRIC = "G elements/s and achieved HBM GB/s (% of B200 peak) for rotate+FP4 quantize"
 SPEC_HBM_GBS = 8000.0
+SM_MAX_HZ = 1.965e9            # B200 maximum SM clock: cycles of the device-side wait per second
 E8, U4, U5 = 0, 1, 2
 NONE, COMP, GIVEN, FROM_AMAX = 0, 1, 2, 3
 
@@ -73,6 +75,11 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: max(3, steps // 20))")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-batch-amax", action="store_true",
+                    help="one fp4q_tensor_amax_accumulate call per tensor instead of one batched amax call "
+                         "per layer group")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="enqueue every timed step call by call instead of replaying it as one CUDA graph")
     ap.add_argument("--separate-mse", action="store_true",
                     help="measure the MSE with its own pass over x (fp4q_quantize + fp4q_block_mse + fp4q_dequantize)")
     ap.add_argument("--separate-dequant", action="store_true",
@@ -214,13 +221,16 @@ def stage_kind(stage: str) -> str:
     return stage.split("@", 1)[0]
 
 
-def launches_of(stage: str, n: int) -> int:
-    """Kernel launches one C-ABI call of `stage` makes on n elements.  The outlier
-    statistics: one histogram pass and a scan below 2^22 elements; above, a
-    sampled pass, the threshold scan, the main pass, a scan, and a pass and a
-    scan that return at once unless the threshold missed."""
+def launches_of(stage: str, n: int, tensors: int = 1) -> int:
+    """Kernel launches one C-ABI call of `stage` makes on n elements of `tensors`
+    tensors.  The outlier statistics: one histogram pass and a scan below 2^22
+    elements; above, a sampled pass, the threshold scan, the main pass, a scan,
+    and a pass and a scan that return at once unless the threshold missed.  The
+    amax of a batch: one launch per 32 tensors."""
     if stage_kind(stage) == "outlier_stats":
         return 6 if n >= (1 << 22) else 2
+    if stage_kind(stage) == "amax":
+        return (tensors + 31) // 32
     return 1
 
 
@@ -234,7 +244,8 @@ class Pipeline:
     """
 
     def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False, search=None,
-                 outlier_p=None, groups=None):
+                 outlier_p=None, groups=None, batch_amax=True):
+        import ctypes
         import torch
         self.fq, self.items, self.device = fq, items, device
         L = fq.lib()
@@ -315,22 +326,39 @@ class Pipeline:
             for j in range(max(len(self.calls[i]) for i in grp)):
                 self.order.extend((i, j) for i in grp if j < len(self.calls[i]))
         assert sorted(self.order) == sorted((i, j) for i in range(len(items)) for j in range(len(self.calls[i])))
+        # the step's calls: as in `order`, except that the amax calls of a group (one
+        # variant's tensors of one layer) are one fp4q_tensor_amax_batched call
+        self.step_calls = []             # (stage, fn, args, item indices)
+        self._keep = []                  # host arrays the batched calls point to
+        for grp in groups:
+            for j in range(max(len(self.calls[i]) for i in grp)):
+                idx = [i for i in grp if j < len(self.calls[i])]
+                kinds = {stage_kind(self.calls[i][j][0]) for i in idx}
+                rots = {items[i][4] for i in idx}
+                if batch_amax and kinds == {"amax"} and len(idx) > 1 and len(rots) == 1:
+                    n = len(idx)
+                    arrs = ((ctypes.c_void_p * n)(*[items[i][1].data_ptr() for i in idx]),
+                            (ctypes.c_int64 * n)(*[items[i][1].shape[0] for i in idx]),
+                            (ctypes.c_int64 * n)(*[items[i][1].shape[1] for i in idx]),
+                            (ctypes.c_void_p * n)(*[self.bufs[i]["gscale"].data_ptr() for i in idx]))
+                    self._keep.append(arrs)
+                    stage = "amax" + (f"@{item_tag(items[idx[0]][0])}" if item_tag(items[idx[0]][0]) else "")
+                    self.step_calls.append((stage, L.fp4q_tensor_amax_batched,
+                                            (n, arrs[0], arrs[1], arrs[2], rots.pop(), arrs[3], 1, sh), idx))
+                else:
+                    self.step_calls.extend((self.calls[i][j][0], self.calls[i][j][1], self.calls[i][j][2], [i])
+                                           for i in idx)
         self.elements = sum(x.numel() for _, x, *_ in items)
-        self.launches_per_step = sum(launches_of(self.calls[i][j][0], items[i][1].numel()) for i, j in self.order)
-        self.events_per_step = 1 + len(self.order)
+        self.launches_per_step = sum(launches_of(stage, sum(items[i][1].numel() for i in idx), len(idx))
+                                     for stage, _, _, idx in self.step_calls)
 
-    def step(self, stream, ev=None):
-        """Enqueue one step; ev = events_per_step timing events or None."""
+    def step(self, stream):
+        """Enqueue one step."""
         bad = 0
         if self.any_comp:
             self.gs_all.zero_()       # the maxima accumulate from 0
-        if ev is not None:
-            ev[0].record(stream)
-        for j, (i, k) in enumerate(self.order):
-            _, fn, args = self.calls[i][k]
+        for _, fn, args, _ in self.step_calls:
             bad |= fn(*args)
-            if ev is not None:
-                ev[j + 1].record(stream)
         if bad:
             raise RuntimeError(f"a C-ABI call returned an error status ({bad})")
 
@@ -344,13 +372,26 @@ class Pipeline:
         if bad:
             raise RuntimeError(f"a C-ABI call returned an error status ({bad})")
 
-    def new_events(self):
-        import torch
-        return [torch.cuda.Event(enable_timing=True) for _ in range(self.events_per_step)]
+    def stages(self):
+        """The step's stages (kernel @ variant) in order of first call."""
+        out = []
+        for stage, *_ in self.step_calls:
+            if stage not in out:
+                out.append(stage)
+        return out
 
-    def stage_times(self, ev):
-        """[(item index, stage, ms)] of one step's events."""
-        return [(i, self.calls[i][k][0], ev[j].elapsed_time(ev[j + 1])) for j, (i, k) in enumerate(self.order)]
+    def run_stage(self, stage):
+        """Enqueue, back to back, every call of one stage of the step (their inputs,
+        [amax, G] included, are those a full step leaves in place)."""
+        bad = 0
+        for st, fn, args, _ in self.step_calls:
+            if st == stage:
+                bad |= fn(*args)
+        if bad:
+            raise RuntimeError(f"a C-ABI call returned an error status ({bad})")
+
+    def stage_calls(self, stage):
+        return [idx for st, _, _, idx in self.step_calls if st == stage]
 
 
 # --------------------------------------------------------------------------- clocks
@@ -802,17 +843,36 @@ def main(argv=None):
     stream.wait_stream(torch.cuda.current_stream())
     pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse,
                     separate_dequant=args.separate_dequant, search=args.search, outlier_p=args.outlier_stats,
-                    groups=groups)
+                    groups=groups, batch_amax=not args.no_batch_amax)
     distinct_bytes = sum(x.numel() * 2 for x in {x.data_ptr(): x for _, x, *_ in items}.values())
     in_l2 = distinct_bytes < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
 
     with torch.cuda.stream(stream):
+        t_host = []
         for _ in range(max(3, args.warmup)):
+            t0 = time.perf_counter()
             pipe.step(stream)
+            t_host.append(time.perf_counter() - t0)
             if flush is not None:
                 flush.zero_()
     torch.cuda.synchronize()
+    host_ms = 1e3 * min(t_host)               # host time to enqueue one step call by call
+
+    # The step as one CUDA graph: the same C-ABI calls, captured once on the launching
+    # stream (programmatic dependent launches become programmatic edges), replayed whole,
+    # so that no host enqueue time sits between the kernels of the timed steps.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            pipe.step(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                graph.replay()
+                if flush is not None:
+                    flush.zero_()
+        torch.cuda.synchronize()
 
     # ---- timed region: K steps with events only at step boundaries (consecutive
     # kernels of a step overlap their launch latency; nothing is recorded between them)
@@ -822,11 +882,14 @@ def main(argv=None):
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
-    kernel_steps = max(1, min(args.steps, max(3, 20000 // pipe.events_per_step)))
+    kernel_steps = max(1, min(args.steps, max(3, 20000 // max(1, len(pipe.step_calls)))))
     with sampler, torch.cuda.stream(stream):
         for k in range(args.steps):
             bounds[k][0].record(stream)
-            pipe.step(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                pipe.step(stream)
             bounds[k][1].record(stream)
             if flush is not None:
                 flush.zero_()         # between timed steps, outside the step's events
@@ -836,19 +899,32 @@ def main(argv=None):
         local_ms = sum(a.elapsed_time(b) for a, b in bounds)
         total_ms = reduce_max(local_ms, device)
 
-        # ---- per-kernel pass (kernel_steps more steps, an event after every C-ABI call
-        # on the launching stream): kernel shares and the dominant kernel's achieved bandwidth
-        events = [pipe.new_events() for _ in range(kernel_steps)]
+        # ---- per-kernel pass: kernel_steps more passes in which every stage (one kernel of
+        # one variant) runs all of its calls of a step back to back between two events on
+        # the launching stream, as they overlap in the step itself (programmatic launches);
+        # its time over its launches is the kernel's device time per launch.  Each pass is
+        # queued behind a device-side wait longer than the host needs to enqueue it, so the
+        # stream never runs dry and every interval is device time, not the host's enqueue.
+        stages = pipe.stages()
+        events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stages]
+                  for _ in range(kernel_steps)]
+        backlog_cycles = int(min(3.0 * host_ms + 2.0, 300.0) * 1e-3 * SM_MAX_HZ)
         for k in range(kernel_steps):
-            pipe.step(stream, events[k])
-            if flush is not None:
-                flush.zero_()
+            torch.cuda._sleep(backlog_cycles)
+            for j, stage in enumerate(stages):
+                events[k][j][0].record(stream)
+                pipe.run_stage(stage)
+                events[k][j][1].record(stream)
+                if flush is not None:
+                    flush.zero_()
         torch.cuda.synchronize()
 
     per_kernel = {}
     for k in range(kernel_steps):
-        for i, stage, ms in pipe.stage_times(events[k]):
-            per_kernel.setdefault(stage, []).append((i, ms))
+        for j, stage in enumerate(stages):
+            calls = pipe.stage_calls(stage)
+            ms = events[k][j][0].elapsed_time(events[k][j][1])
+            per_kernel.setdefault(stage, []).extend((idx, ms / len(calls)) for idx in calls)
     elements_step = pipe.elements
     value = world * elements_step * args.steps / (total_ms / 1e3) / 1e9
 
@@ -859,13 +935,17 @@ def main(argv=None):
     for stage, lst in per_kernel.items():
         tot_ms = sum(t for _, t in lst)
         byts = elems = 0.0
-        for i, t in lst:
-            _, x, fmt, block, rot, gmode = items[i]
-            byts += bytes_per_element(block).get(stage_kind(stage), 0.0) * x.numel()
-            elems += x.numel()
+        launches = 0
+        for idx, t in lst:
+            for i in idx:
+                _, x, fmt, block, rot, gmode = items[i]
+                byts += bytes_per_element(block).get(stage_kind(stage), 0.0) * x.numel()
+                elems += x.numel()
+            launches += launches_of(stage, sum(items[i][1].numel() for i in idx), len(idx))
         step_bytes += byts / kernel_steps
         kernels[stage] = {"ms_per_step": tot_ms / kernel_steps, "share": None,
-                          "launches_per_step": len(lst) / kernel_steps,
+                          "calls_per_step": len(lst) / kernel_steps,
+                          "launches_per_step": launches / kernel_steps,
                           "elements_per_launch": elems / len(lst),
                           "algorithmic_bytes_per_launch": byts / len(lst),
                           "GB_per_s": (byts / 1e9) / (tot_ms / 1e3) if tot_ms > 0 else None}
@@ -915,8 +995,12 @@ def main(argv=None):
                    "l2": "L2 flushed between steps (512 MiB write)" if in_l2 else
                          f"inputs larger than L2 ({distinct_bytes / 1e9:.2f} GB of distinct bf16 input)",
                    "parallelism": f"{world} independent replica(s), no data-path collective",
+                   "launch": "each timed step replayed as one CUDA graph of its C-ABI calls" if graph is not None
+                             else "each timed step enqueued call by call",
                    "timing": "CUDA events at step boundaries on the launching stream (value, ms_per_step); "
-                             f"kernel shares from {kernel_steps} more steps with an event after every call",
+                             f"per-kernel figures from {kernel_steps} more passes that run each stage's calls of a "
+                             "step back to back between two events, behind a device-side wait",
+                   "host_enqueue_ms_per_step": host_ms,
                    "input": "bf16 written by torch's seeded generator on the device"},
         "hbm": {"GB_per_s": step_bytes / 1e9 / (step_ms / 1e3), "bytes_per_step": step_bytes,
                 "frac_of_measured": step_bytes / 1e9 / (step_ms / 1e3) / peak,

@@ -97,11 +97,29 @@ def test_weight_pass_schedule():
     pipe.step(_FakeStream())
     names = [n for n, _ in fq.L.log]
     n_nv = sum(1 for v in bench.WEIGHT_PASS_VARIANTS if v[4] == 1)
-    assert names.count("fp4q_tensor_amax_accumulate") == 9 * n_nv
+    # one batched amax call per NVFP4 layer group, then its three quantizer calls
+    assert names.count("fp4q_tensor_amax_batched") == 3 * n_nv
+    assert names.count("fp4q_tensor_amax_accumulate") == 0
     assert names.count("fp4q_quantize_mse_dequantize") == 36
-    assert pipe.launches_per_step == 36 + 9 * n_nv
-    # within an NVFP4 layer group: three amax calls, then three quantizer calls on the same tensors
-    order = [(bench.stage_kind(pipe.calls[i][k][0]), i) for i, k in pipe.order]
+    assert pipe.launches_per_step == 36 + 3 * n_nv
+    steps = [(bench.stage_kind(st), idx) for st, _, _, idx in pipe.step_calls]
+    nv_first = next(j for j, (kind, _) in enumerate(steps) if kind == "amax")
+    grp = steps[nv_first:nv_first + 4]
+    assert [k for k, _ in grp] == ["amax"] + ["quantize_mse_dequantize"] * 3
+    assert grp[0][1] == [i for _, (i,) in grp[1:]]
+    args = pipe.step_calls[nv_first][2]
+    assert args[0] == 3 and args[6] == 1                       # three tensors, accumulating into zeroed slots
+    assert list(args[3]) == [items[i][1].shape[1] for i in grp[0][1]]
+    assert list(args[5]) == [pipe.bufs[i]["gscale"].data_ptr() for i in grp[0][1]]
+    # the per-tensor form: three amax calls, then three quantizer calls on the same tensors
+    fq2 = _FakeFq()
+    pipe2 = bench.Pipeline(fq2, items, "cpu", _FakeStream(), groups=groups, batch_amax=False)
+    fq2.L.log.clear()
+    pipe2.step(_FakeStream())
+    names2 = [n for n, _ in fq2.L.log]
+    assert names2.count("fp4q_tensor_amax_accumulate") == 9 * n_nv
+    assert pipe2.launches_per_step == 36 + 9 * n_nv
+    order = [(bench.stage_kind(pipe2.calls[i][k][0]), i) for i, k in pipe2.order]
     nv_first = next(j for j, (kind, _) in enumerate(order) if kind == "amax")
     grp = order[nv_first:nv_first + 6]
     assert [k for k, _ in grp] == ["amax"] * 3 + ["quantize_mse_dequantize"] * 3
@@ -109,8 +127,7 @@ def test_weight_pass_schedule():
     # one dequantized-output buffer per input tensor, shared by the variants
     assert len({b["deq"].data_ptr() for b in pipe.bufs}) == 9
     # stage names carry the variant
-    assert {bench.item_tag(lbl) for lbl, *_ in items} == {s.split("@")[1] for i, k in pipe.order
-                                                          for s in [pipe.calls[i][k][0]]}
+    assert {bench.item_tag(lbl) for lbl, *_ in items} == {st.split("@")[1] for st, *_ in pipe.step_calls}
 
 
 def test_weight_pass_and_sweep_defaults():
