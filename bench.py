@@ -224,11 +224,12 @@ def stage_kind(stage: str) -> str:
 def launches_of(stage: str, n: int, tensors: int = 1) -> int:
     """Kernel launches one C-ABI call of `stage` makes on n elements of `tensors`
     tensors.  The outlier statistics: one histogram pass and a scan below 2^22
-    elements; above, a sampled pass, the threshold scan, the main pass, a scan,
-    and a pass and a scan that return at once unless the threshold missed.  The
-    amax of a batch: one launch per 32 tensors."""
+    elements; above, a sampled pass, the threshold scan, the sparse main pass and
+    its shared-histogram twin (one of them returns at once), a scan, and a pass
+    and a scan that return at once unless the threshold missed.  The amax of a
+    batch: one launch per 32 tensors."""
     if stage_kind(stage) == "outlier_stats":
-        return 6 if n >= (1 << 22) else 2
+        return 7 if n >= (1 << 22) else 2
     if stage_kind(stage) == "amax":
         return (tensors + 31) // 32
     return 1

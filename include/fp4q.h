@@ -275,7 +275,11 @@ FP4Q_API size_t fp4q_block_mse_workspace_size(int64_t rows, int64_t cols, int bl
  * histogram pass over x.  Larger tensors get three passes:
  *  - a histogram of a sample of rows sets a threshold below the quantile;
  *  - a pass over x counts only the magnitudes at or above the threshold and
- *    takes the channel maxima;
+ *    takes the channel maxima: a streaming pass that adds each counted
+ *    magnitude to the histogram with a global atomic when the sample puts at
+ *    most 1/64 of the magnitudes there, else a pass with a shared-memory
+ *    histogram per CTA (both are launched; the one not needed returns at
+ *    once);
  *  - a further pass, which returns at once unless the rank turned out to lie
  *    below the threshold, counts the rest.
  * Each pass is followed by a single-CTA scan.  Errors: FP4Q_ERR_SHAPE

@@ -988,9 +988,24 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
     const XRing ring = warp_ring<XRing>(smem_ring);
     // A warp's tiles rise, so its tensors do too: one cursor for the copies issued
-    // ahead and one for the tile being reduced.  Tiles past tile0[count] are never
-    // issued, so both cursors stay below count.
-    int ci = 0, cb = 0, cur = -1;
+    // ahead and one for the tile being reduced, each holding its tensor's tile range
+    // (and source) in registers so that a tile of the same tensor costs one compare.
+    // Tiles past tile0[count] are never issued, so both cursors stay below count.
+    struct Cursor {
+        int c;
+        int64_t t0, t1;
+    };
+    auto seek = [&](Cursor& k, int64_t t) {
+        while (t >= k.t1) {
+            ++k.c;
+            k.t0 = k.t1;
+            k.t1 = p.tile0[k.c + 1];
+        }
+    };
+    Cursor ci{0, 0, p.tile0[1]}, cb{0, 0, p.tile0[1]};
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x[0]);
+    int64_t nbytes = 2 * p.n[0];
+    int src_c = 0, cur = -1;
     float mx = 0.0f;
     uint32_t mb = 0;                                       // max |bf16| pattern, two halves
     auto flush = [&]() {
@@ -1011,15 +1026,19 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
     stream_tiles_with<XRing::NSTAGE>(
         n_tiles, warp, n_warps,
         [&](int64_t t, int s) {
-            while (t >= p.tile0[ci + 1]) ++ci;
-            ring.issue(reinterpret_cast<const uint8_t*>(p.x[ci]), 2 * p.n[ci], (t - p.tile0[ci]) * XRing::TILE_BYTES,
-                       s, lane);
+            seek(ci, t);
+            if (ci.c != src_c) {
+                src_c = ci.c;
+                src = reinterpret_cast<const uint8_t*>(p.x[src_c]);
+                nbytes = 2 * p.n[src_c];
+            }
+            ring.issue(src, nbytes, (t - ci.t0) * XRing::TILE_BYTES, s, lane);
         },
         [&](int64_t t, int s) {
-            while (t >= p.tile0[cb + 1]) ++cb;
-            if (cb != cur) {                                // warp-uniform: the tile is the warp's
+            seek(cb, t);
+            if (cb.c != cur) {                              // warp-uniform: the tile is the warp's
                 if (cur >= 0) flush();
-                cur = cb;
+                cur = cb.c;
             }
             uint32_t w[EPT / 2];
             ring.read(s, 0, w);

@@ -14,7 +14,15 @@
 //     threshold L a safe margin below it;
 //  2. the main pass histograms only magnitudes >= L (a few in a thousand for
 //     P99.9) and takes every channel maximum; the magnitudes below L are then
-//     n minus the histogram's total;
+//     n minus the histogram's total.  When the sample puts at most 1/64 of
+//     the magnitudes at or above L, the main pass is a streaming kernel at
+//     full occupancy (the quantizer's cp.async ring, column stripes so that a
+//     lane keeps its channels' maxima in registers) that adds each counted
+//     magnitude to the global histogram with an atomic (the next launch then
+//     sums its 128-bin bucket totals: atomics on the few buckets that hold
+//     the top magnitudes would serialise); otherwise a pass with a
+//     shared-memory histogram per CTA does it (both launches read a device
+//     flag set by the threshold scan);
 //  3. if rank k falls among the counted magnitudes the answer is exact;
 //     otherwise (L was not below the quantile) a pass gated on a device flag
 //     adds the magnitudes below L, and the scan is repeated on the full
@@ -24,7 +32,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "fp4q_device.cuh"
+#include "fp4q_kernels.cuh"
 #include "fp4q_launch.h"
 
 namespace fp4q {
@@ -38,12 +46,18 @@ constexpr int64_t kDirectElems = int64_t(1) << 22;
 constexpr int64_t kSampleElems = int64_t(1) << 20;   // at least this many in the estimate
 constexpr int kMaxSampleStride = 16;
 
+constexpr int kSparseDiv = 64;                // sparse main pass when <= 1/64 of the sample is >= L
+
 struct StatsCtl {
     uint32_t L;          // magnitudes >= L are counted by the main pass
     uint32_t fallback;   // set when the rank lies below L
+    uint32_t dense;      // set when the sample puts more than 1/kSparseDiv of the magnitudes at or above L
+    uint32_t pad;
 };
 
-enum : int { kAllBins = 0, kFromL = 1, kBelowLIfNeeded = 2 };
+static_assert(sizeof(StatsCtl) == 16, "the workspace holds 16 bytes of control words");
+
+enum : int { kAllBins = 0, kFromL = 1, kBelowLIfNeeded = 2, kFromLIfDense = 3 };
 
 struct StatsParams {
     const uint16_t* x;
@@ -103,7 +117,24 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
     pdl_wait();
     pdl_release();
     uint32_t lo = 0u, hi = (uint32_t)kBins;
-    if (p.mode == kFromL) {
+    if (p.mode == kFromL || p.mode == kFromLIfDense) {
+        if (p.mode == kFromLIfDense && !p.ctl->dense) {
+            // the sparse pass ran: its histogram's bucket totals, 8 buckets per CTA
+            // (a thread per bin), written whole (nothing else has touched them)
+            if (blockIdx.x >= kBuckets / 8) return;
+            __shared__ unsigned long long part[32];
+            const int b = (int)blockIdx.x * 8 + (int)(threadIdx.x >> 7);
+            unsigned long long c = p.hist[128 * b + (threadIdx.x & 127)];
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) c += __shfl_xor_sync(0xffffffffu, c, d);
+            if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+            __syncthreads();
+            if ((threadIdx.x & 127) == 0) {
+                const int w0 = (int)(threadIdx.x >> 5);
+                p.buck[b] = part[w0] + part[w0 + 1] + part[w0 + 2] + part[w0 + 3];
+            }
+            return;
+        }
         lo = p.ctl->L;
     } else if (p.mode == kBelowLIfNeeded) {
         if (!p.ctl->fallback) return;
@@ -154,6 +185,116 @@ __global__ void __launch_bounds__(kStatThreads, 1) outlier_hist_kernel(StatsPara
             if (c) atomicMax(dst + j, c << 16);              // |x| as fp32 bits: orders as integers
         }
     }
+}
+
+// ---- the sparse main pass: magnitudes >= L, global atomics, streaming ring
+// A tile is 4 rows x 256 channels (512 bytes a row): lane l copies and reads
+// the 16-byte chunk of channels 8 l .. 8 l + 7 of each row.  Tiles are numbered
+// column block first; when the number of warps is a multiple of the number of
+// column blocks (the launch picks such a grid when it can) a warp's column
+// block never changes and its lanes' channel maxima stay in registers, else
+// they are flushed whenever it does.
+constexpr int kTopRows = 4;
+using TopRing = Ring<16, kTopRows>;
+
+struct TopParams {
+    const uint16_t* x;
+    int64_t rows, cols;
+    int64_t ncb;                 // 256-channel column blocks
+    unsigned long long* hist;
+    unsigned int* colmax;        // or nullptr
+    const StatsCtl* ctl;
+};
+
+// Tile cursor: the warp's tiles advance by n_warps, i.e. by dcb column blocks and
+// drg row groups (n_warps = drg * ncb + dcb), with no division per tile.
+struct TileCursor {
+    int64_t cb, rg;
+    __device__ __forceinline__ void step(int64_t dcb, int64_t drg, int64_t ncb)
+    {
+        cb += dcb;
+        rg += drg;
+        if (cb >= ncb) {
+            cb -= ncb;
+            ++rg;
+        }
+    }
+};
+
+__device__ __forceinline__ void count_top(const uint32_t (&w)[4], const TopParams& p, uint32_t lo, uint32_t span,
+                                          uint32_t (&cmw)[4])
+{
+    const uint32_t a[4] = {w[0] & 0x7fff7fffu, w[1] & 0x7fff7fffu, w[2] & 0x7fff7fffu, w[3] & 0x7fff7fffu};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cmw[k] = max_u16x2(cmw[k], a[k]);
+    const uint32_t m = max_u16x2(max_u16x2(a[0], a[1]), max_u16x2(a[2], a[3]));
+    if (max(m & 0xffffu, m >> 16) < lo) return;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t v = (k & 1) ? a[k >> 1] >> 16 : a[k >> 1] & 0xffffu;
+        if (v - lo < span) atomicAdd(p.hist + v, 1ull);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) outlier_top_kernel(TopParams p)
+{
+    pdl_wait();
+    pdl_release();
+    if (p.ctl->dense) return;
+    const uint32_t lo = p.ctl->L, span = (uint32_t)kBins - lo;
+    extern __shared__ __align__(128) uint8_t smem_ring[];
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const TopRing ring = warp_ring<TopRing>(smem_ring);
+    const int64_t nrg = (p.rows + kTopRows - 1) / kTopRows;
+    const int64_t n_tiles = p.ncb * nrg;
+    const int64_t dcb = n_warps % p.ncb, drg = n_warps / p.ncb;
+    const int64_t row_bytes = 2 * p.cols;
+    TileCursor ci{warp % p.ncb, warp / p.ncb}, cb{warp % p.ncb, warp / p.ncb};
+    uint32_t cmw[4] = {0u, 0u, 0u, 0u};
+    int64_t cur = -1;
+    auto flush_cols = [&]() {
+        const int64_t c0 = cur * 256 + 8 * lane;
+        if (cur >= 0 && p.colmax && c0 < p.cols) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t c = (j & 1) ? cmw[j >> 1] >> 16 : cmw[j >> 1] & 0xffffu;
+                if (c) atomicMax(p.colmax + c0 + j, c << 16);        // |x| as fp32 bits
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cmw[k] = 0u;
+    };
+    stream_tiles_with<TopRing::NSTAGE>(
+        n_tiles, warp, n_warps,
+        [&](int64_t, int s) {
+            const int64_t col = ci.cb * 256 + 8 * lane, r0 = ci.rg * kTopRows;
+            const uint32_t d = ring.base + (uint32_t)(s * TopRing::TILE_BYTES) + ring.wr[0];
+#pragma unroll
+            for (int h = 0; h < kTopRows; ++h) {
+                const bool ok = col < p.cols && r0 + h < p.rows;   // cols % 8 == 0: a chunk is whole or absent
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x) + (ok ? (r0 + h) * row_bytes + 2 * col : 0);
+                cp_async16(d + (uint32_t)(h * TopRing::SUB_BYTES), src, ok ? 16u : 0u);
+            }
+            ci.step(dcb, drg, p.ncb);
+        },
+        [&](int64_t, int s) {
+            if (cb.cb != cur) {                                      // warp-uniform
+                flush_cols();
+                cur = cb.cb;
+            }
+            const bool col_ok = cb.cb * 256 + 8 * lane < p.cols;
+            const int64_t r0 = cb.rg * kTopRows;
+#pragma unroll
+            for (int h = 0; h < kTopRows; ++h) {
+                uint32_t w[4];
+                ring.read(s, h, w);
+                if (col_ok && r0 + h < p.rows) count_top(w, p, lo, span, cmw);
+            }
+            cb.step(dcb, drg, p.ncb);
+        });
+    flush_cols();
 }
 
 // Histogram scans for the single-CTA kernels.  They read the 256 bucket
@@ -288,9 +429,27 @@ __global__ void __launch_bounds__(kStatThreads) outlier_threshold_kernel(Thresho
     if (plow < 0.0) plow = 0.0;
     const unsigned long long rank = (unsigned long long)floor(plow * (double)ns);
     const int L = rank >= 1 ? bin_at_rank(q.shist, rank, sm) : 0;
-    if (threadIdx.x == 0) {
-        q.ctl->L = (uint32_t)(L > 0 ? L : 0);
-        q.ctl->fallback = 0u;
+    // sample magnitudes below L: the buckets before L's, then L's bucket up to L
+    if (threadIdx.x < 32) {
+        const int l = threadIdx.x;
+        unsigned long long below = 0;
+        if (L > 0) {
+            const int b0 = L & ~127;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int bin = b0 + 4 * l + k;
+                if (bin < L) below += q.shist[bin];
+            }
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) below += __shfl_xor_sync(0xffffffffu, below, d);
+        if (l == 0) {
+            if (L > 0) below += sm.bexcl[L >> 7];
+            const unsigned long long at_or_above = ns - below;
+            q.ctl->L = (uint32_t)(L > 0 ? L : 0);
+            q.ctl->fallback = 0u;
+            q.ctl->dense = (L <= 0 || at_or_above * kSparseDiv > ns) ? 1u : 0u;
+        }
     }
 }
 
@@ -326,6 +485,34 @@ __global__ void __launch_bounds__(kStatThreads) outlier_finalize_kernel(Finalize
         if (b >= 0) q.stats[1] = __uint_as_float((uint32_t)b << 16);
         q.stats[0] = sm.top >= 0 ? __uint_as_float((uint32_t)sm.top << 16) : 0.0f;
     }
+}
+
+// The sparse pass's grid: the resident CTAs, rounded down to a multiple that
+// makes the warp count a multiple of the column blocks when that keeps at least
+// half of them (each warp then keeps one column block).
+cudaError_t launch_top(const uint16_t* x, int64_t rows, int64_t cols, unsigned long long* hist,
+                       unsigned int* colmax, const StatsCtl* ctl, cudaStream_t s)
+{
+    TopParams tp{};
+    tp.x = x;
+    tp.rows = rows;
+    tp.cols = cols;
+    tp.ncb = (cols + 255) / 256;
+    tp.hist = hist;
+    tp.colmax = colmax;
+    tp.ctl = ctl;
+    const int64_t tiles = tp.ncb * ((rows + kTopRows - 1) / kTopRows);
+    int grid = grid_for((const void*)outlier_top_kernel, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
+    // CTAs per whole number of column blocks: ncb / gcd(ncb, kWarps)
+    int64_t a = tp.ncb, b = kWarps;
+    while (b) {
+        const int64_t t = a % b;
+        a = b;
+        b = t;
+    }
+    const int64_t unit = tp.ncb / a;
+    if (unit <= grid && (grid / unit) * unit * 2 >= grid) grid = (int)((grid / unit) * unit);
+    return launch_pdl(outlier_top_kernel, grid, kThreads, kRingBytesPerCta, s, tp);
 }
 
 int hist_grid(StatsParams& prm, int sms)
@@ -405,8 +592,12 @@ cudaError_t launch_outlier_stats(const uint16_t* x, int64_t rows, int64_t cols, 
     if ((e = launch_pdl(outlier_threshold_kernel, 1, kStatThreads, 0, s, ThresholdParams{shist, sbuck, p, ctl})) !=
         cudaSuccess)
         return e;
-    // 2. magnitudes >= L, every channel maximum
-    main.mode = kFromL;
+    // 2. magnitudes >= L, every channel maximum: the sparse streaming pass, or (gated on the
+    //    dense flag) the shared-histogram pass
+    if ((e = launch_top(x, rows, cols, hist, reinterpret_cast<unsigned int*>(col_absmax), ctl, s)) !=
+        cudaSuccess)
+        return e;
+    main.mode = kFromLIfDense;
     if ((e = launch_pdl(outlier_hist_kernel, main_blocks, kStatThreads, kHistSmem, s, main)) != cudaSuccess)
         return e;
     if ((e = launch_pdl(outlier_finalize_kernel, 1, kStatThreads, 0, s, FinalizeParams{hist, hbuck, n, p, stats, ctl, 0})) !=

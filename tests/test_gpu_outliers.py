@@ -78,6 +78,18 @@ def test_sampled_path_shapes(fq, p):
         _check(fq, x, p)
 
 
+@pytest.mark.parametrize("rows,cols", [(2049, 4104), (40, 114944), (8191, 520)])
+@pytest.mark.parametrize("p", [0.999, 0.99])
+def test_sparse_main_pass_column_blocks(fq, rows, cols, p):
+    """The sampled path's streaming main pass works on tiles of 4 rows x 256
+    channels: a partial last column block (4104 = 16 x 256 + 8), a row count
+    that is not a multiple of 4, and 449 column blocks (a prime: the warps'
+    column block changes from tile to tile, so channel maxima are flushed on
+    every change) all stay exact."""
+    x, _ = workloads.student_t_outliers_bf16(rows, cols, seed=rows + cols, n_outlier=min(8, cols))
+    _check(fq, x, p)
+
+
 def test_workspace_reuse_and_no_channels(fq):
     ws = torch.empty((fq.lib().fp4q_outlier_stats_workspace_size(),), dtype=torch.uint8, device="cuda")
     for seed in (1, 2):
