@@ -604,11 +604,19 @@ __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u,
     f32x2 bsum[NB];
 #pragma unroll
     for (int bi = 0; bi < NB; ++bi) bsum[bi] = pk(0.0f, 0.0f);
-    const f32x2 nz2 = pk(nz, nz);                // -0: fma(g, S, -0) is the rounded product fp32(g S)
-    bool anyzero = false;
-    if constexpr (FMT != kE8M0) {
+    // A zero-rounded block (UE scale 0) stores plain 0x0 nibbles, which decode to
+    // +0.  Its quotients y * 0 are zeros that keep y's sign, so its code words are
+    // masked to 0, and its products g * 0 get the addend +0 (which makes them +0),
+    // where every other block's get -0 (fma(g, S, -0) is the rounded product
+    // fp32(g S), sign of zero included): its dequantized values go out as +0 and
+    // each of its errors is y itself.
+    uint32_t zmask[NB];
+    f32x2 zadd[NB];
 #pragma unroll
-        for (int bi = 0; bi < NB; ++bi) anyzero |= sc[bi] == 0.0f;
+    for (int bi = 0; bi < NB; ++bi) {
+        zmask[bi] = (FMT != kE8M0 && sc[bi] == 0.0f) ? 0u : 0xffffffffu;
+        const float a = __uint_as_float(__float_as_uint(nz) & zmask[bi]);
+        zadd[bi] = pk(a, a);
     }
     f32x2 vh[EPT / 4];
 #pragma unroll
@@ -627,7 +635,8 @@ __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u,
                 // hardware E2M1 rounding (nearest, ties to the even code, saturating)
                 const f32x2 R2 = pk(rm[bi], rm[bi]), nS2 = pk(-sc[bi], -sc[bi]);
                 cw[k] = pack_pairs_dec(div2_cr(vk[0], R2, nS2), div2_cr(vk[1], R2, nS2), div2_cr(vk[2], R2, nS2),
-                                       div2_cr(vk[3], R2, nS2), h);
+                                       div2_cr(vk[3], R2, nS2), h) &
+                        zmask[bi];
             } else {
                 // extreme scales: correctly rounded divisions
                 cw[k] = sc[bi] != 0.0f ? pack_pairs_div(vk[0], vk[1], vk[2], vk[3], sc[bi]) : 0u;
@@ -640,14 +649,13 @@ __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u,
             }
         }
         if constexpr (MSE) {
-            // zero-rounded blocks (S = 0) give v = 0 whatever the decoded bytes
             const f32x2 s2 = pk(sc[bi], sc[bi]);
             uint32_t yw[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 __half2 hh = *reinterpret_cast<__half2*>(&h[j]);
                 const f32x2 g = pk(__low2float(hh), __high2float(hh));
-                const f32x2 vq = fma2(g, s2, nz2);                   // v = fp32(g S)
+                const f32x2 vq = fma2(g, s2, zadd[bi]);              // v = fp32(g S); +0 in a zero-rounded block
                 const f32x2 d = sub2(vk[j], vq);                     // y - v
                 bsum[bi] = fma2(d, d, bsum[bi]);
                 if constexpr (DQ) {
@@ -679,22 +687,6 @@ __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u,
             }
         }
     }
-    if constexpr (FMT != kE8M0) {
-        if (anyzero) {
-#pragma unroll
-            for (int k = 0; k < EPT / 8; ++k) {
-                if (sc[(8 * k) / BE] == 0.0f) {
-                    cw[k] = 0u;                                // zero-rounded blocks store plain 0x0 nibbles
-                    if constexpr (DQ) {                        // ... which dequantize to +0
-                        const int64_t ew = u * EPT + 8 * k;
-                        for (int j = 0; j < 8; ++j)
-                            if (ew + j < p.n) p.y[ew + j] = 0u;
-                    }
-                }
-            }
-        }
-    }
-
     if constexpr (MSE) {
         float tot = 0.0f, mx = 0.0f, zr = 0.0f;
 #pragma unroll

@@ -286,12 +286,12 @@ __global__ void __launch_bounds__(kThreads) outlier_top_kernel(TopParams p)
             }
             const bool col_ok = cb.cb * 256 + 8 * lane < p.cols;
             const int64_t r0 = cb.rg * kTopRows;
+            uint32_t w[kTopRows][4];                                 // all four rows' reads in flight at once
 #pragma unroll
-            for (int h = 0; h < kTopRows; ++h) {
-                uint32_t w[4];
-                ring.read(s, h, w);
-                if (col_ok && r0 + h < p.rows) count_top(w, p, lo, span, cmw);
-            }
+            for (int h = 0; h < kTopRows; ++h) ring.read(s, h, w[h]);
+#pragma unroll
+            for (int h = 0; h < kTopRows; ++h)
+                if (col_ok && r0 + h < p.rows) count_top(w[h], p, lo, span, cmw);
             cb.step(dcb, drg, p.ncb);
         });
     flush_cols();
