@@ -78,6 +78,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-batch-amax", action="store_true",
                     help="one fp4q_tensor_amax_accumulate call per tensor instead of one batched amax call "
                          "per layer group")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="weight pass: only the first N of the 48 layers (a smaller case of the same kernels)")
+    ap.add_argument("--no-batch-quantize", action="store_true",
+                    help="one fp4q_quantize_mse_dequantize call per tensor instead of one batched call per layer "
+                         "group (MXFP4 b32 and NVFP4 b16)")
     ap.add_argument("--no-graph", action="store_true",
                     help="enqueue every timed step call by call instead of replaying it as one CUDA graph")
     ap.add_argument("--separate-mse", action="store_true",
@@ -170,6 +175,8 @@ def build_workload(name: str, device, rank: int, args):
         # one bf16 copy of the 48 x 7 weights (26.4 GB); the four variants read it in
         # turn, variant by variant, so each pass streams the whole model from HBM
         sigmas = W.layer_sigmas(W.QWEN25_14B_LAYERS, 0.02, 0.5, rank_seed(14, rank))
+        if args.layers is not None:
+            sigmas = sigmas[:max(1, min(args.layers, len(sigmas)))]    # the first layers (a profiling case)
         xs = []
         for layer, sigma in enumerate(sigmas):
             for ti, t in enumerate(W.QWEN25_14B_LAYER):
@@ -232,6 +239,8 @@ def launches_of(stage: str, n: int, tensors: int = 1) -> int:
         return 7 if n >= (1 << 22) else 2
     if stage_kind(stage) == "amax":
         return (tensors + 31) // 32
+    if stage_kind(stage) == "quantize_mse_dequantize":
+        return (tensors + 7) // 8
     return 1
 
 
@@ -245,7 +254,7 @@ class Pipeline:
     """
 
     def __init__(self, fq, items, device, stream, separate_mse=False, separate_dequant=False, search=None,
-                 outlier_p=None, groups=None, batch_amax=True):
+                 outlier_p=None, groups=None, batch_amax=True, batch_quantize=True):
         import ctypes
         import torch
         self.fq, self.items, self.device = fq, items, device
@@ -336,7 +345,27 @@ class Pipeline:
                 idx = [i for i in grp if j < len(self.calls[i])]
                 kinds = {stage_kind(self.calls[i][j][0]) for i in idx}
                 rots = {items[i][4] for i in idx}
-                if batch_amax and kinds == {"amax"} and len(idx) > 1 and len(rots) == 1:
+                fmts = {(items[i][2], items[i][3], items[i][5]) for i in idx}
+                if (batch_quantize and kinds == {"quantize_mse_dequantize"} and len(idx) > 1 and len(rots) == 1
+                        and len(fmts) == 1 and next(iter(fmts))[:2] in ((E8, 32), (U4, 16))):
+                    # one fp4q_quantize_mse_dequantize_batched call for the group's tensors
+                    n = len(idx)
+                    fmt, block, gmode = next(iter(fmts))
+                    descs = (fq.Fp4qTensor * n)()
+                    for j, i in enumerate(idx):
+                        b, x = self.bufs[i], items[i][1]
+                        descs[j] = fq.Fp4qTensor(x.data_ptr(), x.shape[0], x.shape[1], b["codes"].data_ptr(),
+                                                 b["scales"].data_ptr(),
+                                                 b["gscale"].data_ptr() if gmode == COMP else None,
+                                                 b["deq"].data_ptr(), b["bm"].data_ptr(), b["terms"].data_ptr())
+                    bws = torch.zeros((fq.fp4q_quantize_batch_workspace_size(n),), dtype=torch.uint8, device=device)
+                    self._keep.append((descs, bws))
+                    tag = item_tag(items[idx[0]][0])
+                    stage = "quantize_mse_dequantize" + (f"@{tag}" if tag else "")
+                    self.step_calls.append((stage, L.fp4q_quantize_mse_dequantize_batched,
+                                            (n, descs, fmt, block, rots.pop(), FROM_AMAX if gmode == COMP else NONE,
+                                             bws.data_ptr(), bws.numel(), sh), idx))
+                elif batch_amax and kinds == {"amax"} and len(idx) > 1 and len(rots) == 1:
                     n = len(idx)
                     arrs = ((ctypes.c_void_p * n)(*[items[i][1].data_ptr() for i in idx]),
                             (ctypes.c_int64 * n)(*[items[i][1].shape[0] for i in idx]),
@@ -844,7 +873,8 @@ def main(argv=None):
     stream.wait_stream(torch.cuda.current_stream())
     pipe = Pipeline(fq, items, device, stream, separate_mse=args.separate_mse,
                     separate_dequant=args.separate_dequant, search=args.search, outlier_p=args.outlier_stats,
-                    groups=groups, batch_amax=not args.no_batch_amax)
+                    groups=groups, batch_amax=not args.no_batch_amax,
+                    batch_quantize=not args.no_batch_quantize)
     distinct_bytes = sum(x.numel() * 2 for x in {x.data_ptr(): x for _, x, *_ in items}.values())
     in_l2 = distinct_bytes < 256 * 2 ** 20
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if in_l2 else None
@@ -988,6 +1018,7 @@ def main(argv=None):
                    "variants": tags if tags != [""] else None,
                    "format": describe_format(items),
                    "rot": sorted({it[4] for it in items}), "elements_per_step": elements_step,
+                   "layers": (args.layers or 48) if args.workload == "qwen25_14b_weight_pass" else None,
                    "distinct_input_bytes": distinct_bytes,
                    "block_scales": "max rule" if args.search is None else
                                    f"MSE search: max-rule code, {args.search[1]} above, {args.search[0]} below",

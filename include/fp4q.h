@@ -134,6 +134,45 @@ FP4Q_API int fp4q_quantize_search(const void* x, int64_t rows, int64_t cols, int
                                   float* gscale, void* stream);
 
 /*
+ * fp4q_quantize_mse_dequantize_batched -- fp4q_quantize_mse_dequantize for
+ * `count` tensors of one format, block and rotation (a model layer's
+ * projections), in one launch per 8 tensors.  The tensors' tiles are laid end
+ * to end and streamed by one kernel, so small tensors cost no launch ramp and
+ * tail of their own.  Each tensor keeps its own per-tensor scale, outputs and
+ * MSE terms, bit for bit those of the single call ("Finer is better?",
+ * Theoretical framework; "Diagnosing FP4 inference", Methodology: quantized
+ * on the fly, then dequantized for the compute).
+ *  tensors    host array of `count` descriptors, read during the call only;
+ *             per tensor the arguments of fp4q_quantize_mse_dequantize, with
+ *             the same layouts, alignment and meaning (y required).
+ *  fmt, block FP4Q_SCALE_E8M0 with block 32 (MXFP4) or FP4Q_SCALE_UE4M3 with
+ *             block 16 (NVFP4); other pairs: FP4Q_ERR_UNSUPPORTED (use the
+ *             single call).
+ *  rot, gmode as for fp4q_quantize (E8M0: FP4Q_GLOBAL_NONE only).
+ *  workspace  device scratch of fp4q_quantize_batch_workspace_size(count)
+ *             bytes (8-byte aligned), zero-filled before its first use and
+ *             left so by every call: tensor i uses slice i (a completion
+ *             counter and per-CTA partials).
+ * Every tensor is checked before anything is enqueued; errors as for
+ * fp4q_quantize_mse_dequantize, FP4Q_ERR_SHAPE for count < 0 (count = 0 does
+ * nothing).
+ */
+typedef struct fp4q_tensor {
+    const void* x;       /* bf16 [rows][cols] (device, 32-byte aligned) */
+    int64_t rows, cols;
+    uint8_t* codes;      /* rows*cols/2 bytes (32-byte aligned) */
+    uint8_t* scales;     /* rows*cols/block bytes (16-byte aligned) */
+    float* gscale;       /* per gmode, as fp4q_quantize; NULL for FP4Q_GLOBAL_NONE */
+    void* y;             /* bf16 [rows][cols] dequantized values (32-byte aligned) */
+    float* block_mse;    /* rows*cols/block floats (16-byte aligned) or NULL */
+    double* terms;       /* 4 doubles: total, non-max, max, zero-rounded MSE (8-byte aligned) */
+} fp4q_tensor;
+FP4Q_API size_t fp4q_quantize_batch_workspace_size(int count);
+FP4Q_API int fp4q_quantize_mse_dequantize_batched(int count, const fp4q_tensor* tensors, int fmt, int block,
+                                                  int rot, int gmode, void* workspace, size_t ws_bytes,
+                                                  void* stream);
+
+/*
  * fp4q_tensor_amax -- amax = max |y| over the whole (optionally rotated)
  * tensor, written as one float.  This is the first half of the per-tensor
  * scale of COMPUTE mode ("Finer is better?", Results: UE4M3 with a dynamic

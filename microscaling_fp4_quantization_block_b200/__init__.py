@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
         "fp4q_tensor_amax": (I, [P, I64, I64, I, P, P]),
         "fp4q_tensor_amax_accumulate": (I, [P, I64, I64, I, P, P]),
         "fp4q_tensor_amax_batched": (I, [I, P, P, P, I, P, I, P]),
+        "fp4q_quantize_batch_workspace_size": (SZ, [I]),
+        "fp4q_quantize_mse_dequantize_batched": (I, [I, P, I, I, I, I, P, SZ, P]),
         "fp4q_global_scale": (I, [P, P, P]),
         "fp4q_dequantize": (I, [P, P, P, I64, I64, I, I, I, I, P, P]),
         "fp4q_block_mse": (I, [P, P, P, P, I64, I64, I, I, I, P, P, P, SZ, P]),
@@ -493,6 +495,55 @@ def fp4q_quantize_mse_dequantize(x: torch.Tensor, fmt, block: int, rot: int = 0,
                                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "fp4q_quantize_mse_dequantize")
     return codes, scales, gscale, y, block_mse, terms
+
+
+class Fp4qTensor(ctypes.Structure):
+    """One tensor of a batched call (include/fp4q.h: fp4q_tensor)."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("gscale", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("block_mse", ctypes.c_void_p), ("terms", ctypes.c_void_p)]
+
+
+def fp4q_quantize_batch_workspace_size(count: int) -> int:
+    return lib().fp4q_quantize_batch_workspace_size(count)
+
+
+def fp4q_quantize_mse_dequantize_batched(xs, fmt, block: int, rot: int = 0, gmode="none", gscales=None,
+                                         want_block_mse: bool = True, workspace: Optional[torch.Tensor] = None,
+                                         stream=None):
+    """fp4q_quantize_mse_dequantize for every tensor of xs in one pass (MXFP4 b32
+    or NVFP4 b16): a list of (codes, scales, gscale, y, block_mse, terms).
+    gscales: per-tensor gscale buffers (FROM_AMAX: [amax, G] each), else allocated."""
+    xs = [x.contiguous() for x in xs]
+    for x in xs:
+        if x.dtype != torch.bfloat16 or x.dim() != 2:
+            raise ValueError("every x must be a 2-D bf16 tensor")
+    _need_cuda(*xs)
+    fmt, gmode = _fmt(fmt), _gmode(gmode)
+    if gmode == FP4Q_GLOBAL_FROM_AMAX and gscales is None:
+        raise ValueError("from_amax mode reads each tensor maximum from gscale[0]: pass 2-float gscales")
+    n = len(xs)
+    dev = xs[0].device if xs else torch.device("cuda")
+    outs, descs = [], (Fp4qTensor * max(n, 1))()
+    for i, x in enumerate(xs):
+        rows, cols = x.shape
+        g = gscales[i] if gscales is not None else (
+            torch.empty((1,), dtype=torch.float32, device=dev) if gmode != FP4Q_GLOBAL_NONE else None)
+        o = (torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+             torch.empty((rows, cols // block), dtype=torch.uint8, device=dev), g,
+             torch.empty((rows, cols), dtype=torch.bfloat16, device=dev),
+             torch.empty((rows, cols // block), dtype=torch.float32, device=dev) if want_block_mse else None,
+             torch.empty((4,), dtype=torch.float64, device=dev))
+        _need_cuda(*[t for t in o if t is not None])
+        descs[i] = Fp4qTensor(_ptr(x), rows, cols, _ptr(o[0]), _ptr(o[1]), _ptr(o[2]), _ptr(o[3]), _ptr(o[4]),
+                              _ptr(o[5]))
+        outs.append(o)
+    if workspace is None:
+        workspace = torch.zeros((max(1, fp4q_quantize_batch_workspace_size(n)),), dtype=torch.uint8, device=dev)
+    st = lib().fp4q_quantize_mse_dequantize_batched(n, descs, fmt, block, rot, gmode, _ptr(workspace),
+                                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "fp4q_quantize_mse_dequantize_batched")
+    return outs
 
 
 def fp4q_e2m1_encode_f32(r: torch.Tensor, packed: Optional[torch.Tensor] = None,

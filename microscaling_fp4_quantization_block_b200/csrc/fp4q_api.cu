@@ -341,6 +341,88 @@ int fp4q_quantize_mse_dequantize(const void* x, int64_t rows, int64_t cols, int 
                              workspace, ws_bytes, stream);
 }
 
+// Per-tensor slice of the batched quantizer's workspace: the completion counter,
+// then kMaxPartialCtas partial slots of 4 doubles.
+constexpr size_t kBatchSliceBytes = kCounterBytes + (size_t)kMaxPartialCtas * 4 * sizeof(double);
+
+size_t fp4q_quantize_batch_workspace_size(int count)
+{
+    return count > 0 ? (size_t)count * kBatchSliceBytes : 0;
+}
+
+int fp4q_quantize_mse_dequantize_batched(int count, const fp4q_tensor* tensors, int fmt, int block, int rot,
+                                         int gmode, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (count < 0) return FP4Q_ERR_SHAPE;
+    if (count == 0) return FP4Q_OK;
+    if (!tensors || !workspace) return FP4Q_ERR_NULL;
+    if (!((fmt == FP4Q_SCALE_E8M0 && block == 32) || (fmt == FP4Q_SCALE_UE4M3 && block == 16)))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!valid_gmode(gmode)) return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_SCALE_E8M0 && gmode != FP4Q_GLOBAL_NONE) return FP4Q_ERR_UNSUPPORTED;
+    if (!aligned(workspace, 8)) return FP4Q_ERR_ALIGN;
+    if (ws_bytes < fp4q_quantize_batch_workspace_size(count)) return FP4Q_ERR_WORKSPACE;
+    for (int i = 0; i < count; ++i) {                  // every tensor checked before anything is enqueued
+        const fp4q_tensor& t = tensors[i];
+        int64_t n = 0;
+        int st = check_shape(t.rows, t.cols, fmt, block, rot, &n);
+        if (st) return st;
+        if (!t.terms) return FP4Q_ERR_NULL;
+        if (!aligned(t.terms, 8)) return FP4Q_ERR_ALIGN;
+        if (gmode != FP4Q_GLOBAL_NONE) {
+            if (!t.gscale) return FP4Q_ERR_NULL;
+            if (!aligned(t.gscale, 4)) return FP4Q_ERR_ALIGN;
+        }
+        if (n > 0) {
+            if (!t.x || !t.codes || !t.scales || !t.y) return FP4Q_ERR_NULL;
+            if (!aligned(t.x, 32) || !aligned(t.codes, 32) || !aligned(t.scales, 16) || !aligned(t.y, 32))
+                return FP4Q_ERR_ALIGN;
+        }
+        if (t.block_mse && !aligned(t.block_mse, 16)) return FP4Q_ERR_ALIGN;
+        if (n > (int64_t)(INT32_MAX / kQuantBatch) * kAmaxTileElems) return FP4Q_ERR_SHAPE;   // tile indices fit 32 bits
+    }
+    cudaStream_t s = as_stream(stream);
+    if (gmode == FP4Q_GLOBAL_COMPUTE) {
+        // the tensors' maxima, then G = amax / 2688 in place; the quantizer reads G as given
+        for (int i = 0; i < count; ++i) {
+            const fp4q_tensor& t = tensors[i];
+            cudaError_t e = enqueue_amax(t.x, t.rows * t.cols, rot, t.gscale, s);
+            if (e == cudaSuccess) {
+                global_scale_kernel<<<1, 1, 0, s>>>(t.gscale, t.gscale);
+                e = cudaGetLastError();
+            }
+            if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+        }
+    }
+    char* ws = static_cast<char*>(workspace);
+    for (int c0 = 0; c0 < count; c0 += kQuantBatch) {
+        QuantBatchParams bp{};
+        bp.count = count - c0 < kQuantBatch ? count - c0 : kQuantBatch;
+        bp.tile0[0] = 0;
+        for (int j = 0; j < bp.count; ++j) {
+            const fp4q_tensor& t = tensors[c0 + j];
+            QuantParams& q = bp.t[j];
+            q.x = static_cast<const uint16_t*>(t.x);
+            q.n = t.rows * t.cols;
+            q.codes = t.codes;
+            q.scales = t.scales;
+            set_global(gmode == FP4Q_GLOBAL_COMPUTE ? FP4Q_GLOBAL_GIVEN : gmode, t.gscale, &q.gsrc, &q.gdst);
+            q.block_mse = t.block_mse;
+            void* slice = ws + (size_t)(c0 + j) * kBatchSliceBytes;
+            q.partials = mse_partials(slice);
+            q.done = mse_counter(slice);
+            q.terms = t.terms;
+            q.y = static_cast<uint16_t*>(t.y);
+            rotation_constants(rot, &q.c_hi, &q.c_lo);
+            bp.tile0[j + 1] = bp.tile0[j] + (int32_t)((q.n + kAmaxTileElems - 1) / kAmaxTileElems);
+        }
+        cudaError_t e = fmt == FP4Q_SCALE_E8M0 ? launch_quantize_batch_e8m0(block, rot, bp, s)
+                                               : launch_quantize_batch_ue4m3(block, rot, bp, s);
+        if (e != cudaSuccess) return FP4Q_ERR_CUDA;
+    }
+    return FP4Q_OK;
+}
+
 int fp4q_tensor_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax, void* stream)
 {
     int64_t n = 0;

@@ -140,10 +140,11 @@ __device__ __forceinline__ R warp_ring(uint8_t* smem)
 
 // Ring pipeline driver: calls body(tile, stage) for every tile of this warp,
 // with the tile's input resident in the ring; issue(tile, stage) starts the
-// copies of a tile.  NSTAGE - 1 tiles are in flight.
-template <int NS, typename Issue, typename Body>
-__device__ __forceinline__ void stream_tiles_with(int64_t n_tiles, int64_t warp, int64_t n_warps, Issue&& issue,
-                                                  Body&& body)
+// copies of a tile.  NSTAGE - 1 tiles are in flight.  ring_prime issues the
+// first NSTAGE - 1 tiles, ring_run the rest while it runs the body: a kernel can
+// prime its ring first and overlap the copies' latency with its own set-up.
+template <int NS, typename Issue>
+__device__ __forceinline__ void ring_prime(int64_t n_tiles, int64_t warp, int64_t n_warps, Issue&& issue)
 {
     int64_t t_issue = warp;
 #pragma unroll
@@ -152,6 +153,12 @@ __device__ __forceinline__ void stream_tiles_with(int64_t n_tiles, int64_t warp,
         cp_async_commit();
         t_issue += n_warps;
     }
+}
+
+template <int NS, typename Issue, typename Body>
+__device__ __forceinline__ void ring_run(int64_t n_tiles, int64_t warp, int64_t n_warps, Issue&& issue, Body&& body)
+{
+    int64_t t_issue = warp + (int64_t)(NS - 1) * n_warps;
     int stage = 0;
     for (int64_t t = warp; t < n_tiles; t += n_warps) {
         const int s_new = stage == 0 ? NS - 1 : stage - 1;          // the slot read last iteration
@@ -165,6 +172,14 @@ __device__ __forceinline__ void stream_tiles_with(int64_t n_tiles, int64_t warp,
         __syncwarp();                                              // slot may be refilled next iteration
     }
     cp_async_wait_all();
+}
+
+template <int NS, typename Issue, typename Body>
+__device__ __forceinline__ void stream_tiles_with(int64_t n_tiles, int64_t warp, int64_t n_warps, Issue&& issue,
+                                                  Body&& body)
+{
+    ring_prime<NS>(n_tiles, warp, n_warps, issue);
+    ring_run<NS>(n_tiles, warp, n_warps, issue, body);
 }
 
 // The same over one contiguous input of nbytes bytes, tile t at byte t * TILE_BYTES.
@@ -526,7 +541,8 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_
 // Store a unit's code word (16 bytes; with EF evict-first in L2, for codes
 // that nothing reads again in the step) and its blocks' scale bytes; a unit
 // that reaches past n stores only its valid prefix.
-template <int B, int K, bool EF>
+// SF = false: the caller never asks for the block-scaled MMA layout (sf_cols = 0).
+template <int B, int K, bool EF, bool SF = true>
 __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, const uint32_t (&cw)[EPT / 8],
                                            const uint32_t (&code)[UnitShape<B, K>::NB], int lane, uint64_t pol)
 {
@@ -546,7 +562,7 @@ __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, cons
             for (int j = 0; j < 4; ++j)
                 if (4 * k + j < nbytes) cdst[4 * k + j] = (uint8_t)(cw[k] >> (8 * j));
     }
-    if (p.sf_cols > 0) {
+    if (SF && p.sf_cols > 0) {
         // the block-scaled MMA layout: a unit's blocks lie in one row
         const int64_t g0 = e0 / B;
         const int64_t r = g0 / p.sf_cols, j0 = g0 - r * p.sf_cols;
@@ -584,7 +600,7 @@ __device__ __forceinline__ void store_unit(const QuantParams& p, int64_t u, cons
 // blocks' absolute maxima are m and whose (rotated) values are produced half
 // by half: half(h, vh) fills vh with elements 16 h .. 16 h + 15 as 8 pairs
 // (h = 0 then 1), so a caller can hold only half of the unit in registers.
-template <int FMT, int B, int K, bool MSE, bool DQ, typename Half>
+template <int FMT, int B, int K, bool MSE, bool DQ, bool SF = true, typename Half>
 __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u, Half&& half,
                                                 const float (&m)[UnitShape<B, K>::NB], int lane,
                                                 const ScaleConsts& kc, const float2* tab, float nz,
@@ -715,17 +731,17 @@ __device__ __forceinline__ void quantize_halves(const QuantParams& p, int64_t u,
     }
 
     // ---- stores
-    store_unit<B, K, DQ>(p, u, cw, code, lane, pol);
+    store_unit<B, K, DQ, SF>(p, u, cw, code, lane, pol);
 }
 
 // The same for a unit held whole in registers.
-template <int FMT, int B, int K, bool MSE, bool DQ>
+template <int FMT, int B, int K, bool MSE, bool DQ, bool SF = true>
 __device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u, const f32x2 (&v)[EPT / 2],
                                                 const float (&m)[UnitShape<B, K>::NB], int lane,
                                                 const ScaleConsts& kc, const float2* tab, float nz,
                                                 double (&acc)[3], uint64_t pol)
 {
-    quantize_halves<FMT, B, K, MSE, DQ>(
+    quantize_halves<FMT, B, K, MSE, DQ, SF>(
         p, u,
         [&](int h, f32x2 (&vh)[EPT / 4]) {
 #pragma unroll
@@ -734,18 +750,28 @@ __device__ __forceinline__ void quantize_values(const QuantParams& p, int64_t u,
         m, lane, kc, tab, nz, acc, pol);
 }
 
+// SF as for store_unit; c_hi, c_lo: the rotation constant (p's own, or one a
+// batch of tensors shares).
+template <int FMT, int B, int K, bool MSE, bool DQ, bool SF = true>
+__device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
+                                              int lane, const ScaleConsts& kc, const float2* tab, float nz,
+                                              double (&acc)[3], uint64_t pol, float c_hi, float c_lo)
+{
+    using S = UnitShape<B, K>;
+    f32x2 v[EPT / 2];
+    load_unit<K>(w, v, lane, c_hi, c_lo);
+    float m[S::NB];
+    if constexpr (K == 0) block_max_words<B>(w, m);
+    else block_max<B, K>(v, m);
+    quantize_values<FMT, B, K, MSE, DQ, SF>(p, u, v, m, lane, kc, tab, nz, acc, pol);
+}
+
 template <int FMT, int B, int K, bool MSE, bool DQ>
 __device__ __forceinline__ void quantize_unit(const QuantParams& p, int64_t u, const uint32_t (&w)[EPT / 2],
                                               int lane, const ScaleConsts& kc, const float2* tab, float nz,
                                               double (&acc)[3], uint64_t pol)
 {
-    using S = UnitShape<B, K>;
-    f32x2 v[EPT / 2];
-    load_unit<K>(w, v, lane, p.c_hi, p.c_lo);
-    float m[S::NB];
-    if constexpr (K == 0) block_max_words<B>(w, m);
-    else block_max<B, K>(v, m);
-    quantize_values<FMT, B, K, MSE, DQ>(p, u, v, m, lane, kc, tab, nz, acc, pol);
+    quantize_unit<FMT, B, K, MSE, DQ, true>(p, u, w, lane, kc, tab, nz, acc, pol, p.c_hi, p.c_lo);
 }
 
 // Two CTAs per SM (up to 128 registers) unless the kernel fits three without
@@ -762,6 +788,18 @@ __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quant
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
     const XRing ring = warp_ring<XRing>(smem_ring);
+
+    // Evict-first in L2 for what the step does not read again, so that it does
+    // not push out lines that are: x where this is its last read (MSE fused), and
+    // the codes and dequantized values of the fused dequantizing kernel.
+    const uint64_t pol = l2_evict_first();
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x);
+    auto issue = [&](int64_t t, int s) { ring.template issue<MSE>(src, 2 * p.n, t * XRing::TILE_BYTES, s, lane, pol); };
+    // The first tiles load during the set-up below, except in the rotated UE-scale
+    // kernels: their loop is the most register-bound, and starting the copies
+    // earlier measured 2.5% slower there (1-2% faster elsewhere).
+    constexpr bool kPrimeEarly = FMT == kE8M0 || K == 0;
+    if constexpr (kPrimeEarly) ring_prime<XRing::NSTAGE>(n_tiles, warp, n_warps, issue);
 
     float G = 1.0f;
     if (FMT != kE8M0 && p.gsrc != nullptr) {
@@ -782,21 +820,185 @@ __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quant
     const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
     double acc[3] = {0.0, 0.0, 0.0};        // squared errors: all, block maxima, zero-rounded blocks
 
-    // Evict-first in L2 for what the step does not read again, so that it does
-    // not push out lines that are: x where this is its last read (MSE fused), and
-    // the codes and dequantized values of the fused dequantizing kernel.
-    const uint64_t pol = l2_evict_first();
-    stream_tiles<MSE>(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
-                            [&](int64_t t, int s) {
-                                uint32_t w[EPT / 2];
-                                ring.read(s, 0, w);
-                                quantize_unit<FMT, B, K, MSE, DQ>(p, t * 32 + lane, w, lane, kc, tab, nz, acc, pol);
-                            },
-                            pol);
+    if constexpr (!kPrimeEarly) ring_prime<XRing::NSTAGE>(n_tiles, warp, n_warps, issue);
+    ring_run<XRing::NSTAGE>(n_tiles, warp, n_warps, issue, [&](int64_t t, int s) {
+        uint32_t w[EPT / 2];
+        ring.read(s, 0, w);
+        quantize_unit<FMT, B, K, MSE, DQ>(p, t * 32 + lane, w, lane, kc, tab, nz, acc, pol);
+    });
     if constexpr (MSE) {
         cta_partials(acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2], p.partials);
         finish_partials(p.partials, p.done, p.n, p.terms);
     }
+}
+
+// ---------------------------------------------------------------- batched fused quantizer
+// One launch quantizes up to kQuantBatch tensors of one format, block and
+// rotation, each with its own per-tensor scale, outputs and MSE terms (what
+// fp4q_quantize_mse_dequantize does for one).  Their ring tiles are laid end
+// to end and every warp strides over all of them, so a layer's small
+// projections pay one launch ramp and one tail instead of one each.
+constexpr int kQuantBatch = 8;
+
+struct QuantBatchParams {
+    QuantParams t[kQuantBatch];          // per tensor: x, n, outputs, gsrc/gdst, partials, done, terms, y
+    int32_t tile0[kQuantBatch + 1];      // first ring tile of each tensor; tile0[count] = all tiles
+    int count;
+};
+
+// The last CTA to finish tensor c (a counter per tensor) sums its per-CTA
+// partials in index order (deterministic) into terms[c] = sum / n.  Every CTA
+// writes a partial for every tensor, zeros for tensors it never touched.
+template <int NT = kThreads>
+__device__ __forceinline__ void finish_partials_batch(const QuantBatchParams& P)
+{
+    constexpr int NW = NT / 32;
+    __shared__ bool last[kQuantBatch];
+    __shared__ double red[NW][4];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x < (unsigned)P.count)
+        last[threadIdx.x] = atomicInc(P.t[threadIdx.x].done, gridDim.x - 1u) == gridDim.x - 1u;
+    __syncthreads();
+    for (int c = 0; c < P.count; ++c) {
+        if (!last[c]) continue;                                    // CTA-uniform
+        __threadfence();
+        const double* partials = P.t[c].partials;
+        double s[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int i = threadIdx.x; i < (int)gridDim.x; i += NT)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[k] += __ldcg(partials + (int64_t)i * 4 + k);
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], d);
+        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+        if (lane == 0)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) red[wid][k] = s[k];
+        __syncthreads();
+        if (threadIdx.x < 4) {
+            double t = 0.0;
+            for (int w = 0; w < NW; ++w) t += red[w][threadIdx.x];
+            P.t[c].terms[threadIdx.x] = P.t[c].n > 0 ? t / (double)P.t[c].n : 0.0;
+        }
+        __syncthreads();
+    }
+}
+
+template <int FMT, int B, int K>
+__global__ void __launch_bounds__(kThreads, 2) quantize_batch_kernel(const __grid_constant__ QuantBatchParams P)
+{
+    pdl_wait();
+    pdl_release();
+    extern __shared__ __align__(128) uint8_t smem_ring[];
+    __shared__ float2 tabs[FMT == kE8M0 ? 1 : kQuantBatch][256];   // UE scales {S, 1/S} by code, per tensor
+    __shared__ float4 kcs[kQuantBatch];                            // per tensor: G, fp32(6G), 1/fp32(6G), in range
+    __shared__ double wsum[kQuantBatch][kWarps][4];                // per tensor and warp: the MSE terms
+    const int lane = threadIdx.x & 31;
+    const int warp_in = threadIdx.x >> 5;
+    const int32_t n_tiles = P.tile0[P.count];
+    const int32_t warp = (int32_t)(blockIdx.x * (kThreads / 32)) + warp_in;
+    const int32_t n_warps = (int32_t)(gridDim.x * (kThreads / 32));
+    const XRing ring = warp_ring<XRing>(smem_ring);
+    const uint64_t pol = l2_evict_first();
+
+    // ---- the tiles of all tensors; a warp's tiles rise, so its tensors do too:
+    // one cursor for the copies issued ahead, one for the tile being quantized
+    struct Cursor {
+        int c;
+        int32_t t0, t1;
+    };
+    auto seek = [&](Cursor& k, int32_t t) {
+        while (t >= k.t1) {
+            ++k.c;
+            k.t0 = k.t1;
+            k.t1 = P.tile0[k.c + 1];
+        }
+    };
+    Cursor ci{0, 0, P.tile0[1]}, cb{0, 0, P.tile0[1]};
+    auto issue = [&](int64_t t, int s) {
+        seek(ci, (int32_t)t);
+        const QuantParams& q = P.t[ci.c];
+        ring.template issue<true>(reinterpret_cast<const uint8_t*>(q.x), 2 * q.n,
+                                  (int64_t)((int32_t)t - ci.t0) * XRing::TILE_BYTES, s, lane, pol);
+    };
+    // the first tiles load during the set-up, except in the rotated UE-scale kernels (as quantize_kernel)
+    constexpr bool kPrimeEarly = FMT == kE8M0 || K == 0;
+    if constexpr (kPrimeEarly) ring_prime<XRing::NSTAGE>(n_tiles, warp, n_warps, issue);
+
+    // ---- per-tensor set-up: G (from the tensor maximum in FROM_AMAX mode), the
+    // scale constants and the UE scale table, and zeroed MSE slots
+    for (int c = 0; c < P.count; ++c) {
+        float G = 1.0f;
+        if (FMT != kE8M0 && P.t[c].gsrc != nullptr) {
+            G = *P.t[c].gsrc;
+            if (P.t[c].gdst != nullptr) {
+                G = G > 0.0f ? __fdiv_rn(G, 2688.0f) : 1.0f;
+                if (blockIdx.x == 0 && threadIdx.x == 0) *P.t[c].gdst = G;
+            }
+        }
+        if (threadIdx.x == 0) {
+            const ScaleConsts k = scale_consts(G);
+            kcs[c] = make_float4(k.G, k.denom, k.rdenom, k.denom_ok ? 1.0f : 0.0f);
+        }
+        if constexpr (FMT != kE8M0) fill_scale_table<FMT>(tabs[c], G);
+    }
+    for (int i = threadIdx.x; i < kQuantBatch * kWarps * 4; i += kThreads) (&wsum[0][0][0])[i] = 0.0;
+    __syncthreads();
+    // -0.0f from a value the compiler cannot see (the tile count is >= 0)
+    const float nz = __uint_as_float(0x80000000u | ((uint32_t)n_tiles >> 31));
+
+    int cur = -1;
+    ScaleConsts kc{};
+    double acc[3] = {0.0, 0.0, 0.0};
+    auto flush = [&]() {                                           // warp-uniform
+        double a[4] = {acc[0], acc[0] - acc[1] - acc[2], acc[1], acc[2]};
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) a[k] += __shfl_xor_sync(0xffffffffu, a[k], d);
+        if (lane == 0)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) wsum[cur][warp_in][k] = a[k];
+        acc[0] = acc[1] = acc[2] = 0.0;
+    };
+    if constexpr (!kPrimeEarly) ring_prime<XRing::NSTAGE>(n_tiles, warp, n_warps, issue);
+    ring_run<XRing::NSTAGE>(n_tiles, warp, n_warps, issue, [&](int64_t t, int s) {
+        seek(cb, (int32_t)t);
+        if (cb.c != cur) {                                         // warp-uniform: the tile is the warp's
+            if (cur >= 0) flush();
+            cur = cb.c;
+            const float4 k4 = kcs[cur];
+            kc.G = k4.x;
+            kc.denom = k4.y;
+            kc.rdenom = k4.z;
+            kc.denom_ok = k4.w != 0.0f;
+        }
+        uint32_t w[EPT / 2];
+        ring.read(s, 0, w);
+        // Every tensor of a batch shares the rotation, and none asks for the MMA scale
+        // layout.  The rotated UE-scale kernels take both as compile-time facts (the
+        // constant from the first entry, no layout test): measured 5% faster there.
+        // The others read them per tensor, which measured 1-3% faster for them: in
+        // these register-bound loops the allocation, not the instruction count,
+        // decides.
+        constexpr bool kShared = FMT != kE8M0 && K != 0;
+        const QuantParams& q = P.t[kShared ? 0 : cur];
+        quantize_unit<FMT, B, K, true, true, !kShared>(P.t[cur], (int64_t)((int32_t)t - cb.t0) * 32 + lane, w,
+                                                       lane, kc, tabs[FMT == kE8M0 ? 0 : cur], nz, acc, pol,
+                                                       q.c_hi, q.c_lo);
+    });
+    if (cur >= 0) flush();
+    __syncthreads();
+    // per-CTA partials of every tensor, warps summed in index order
+    if (threadIdx.x < (unsigned)(P.count * 4)) {
+        const int c = threadIdx.x >> 2, k = threadIdx.x & 3;
+        double sum = 0.0;
+        for (int w = 0; w < kWarps; ++w) sum += wsum[c][w][k];
+        P.t[c].partials[(int64_t)blockIdx.x * 4 + k] = sum;
+    }
+    finish_partials_batch(P);
 }
 
 // ---------------------------------------------------------------- MSE-optimised block scales

@@ -7,6 +7,7 @@
 namespace fp4q {
 
 struct QuantParams;
+struct QuantBatchParams;
 struct AmaxParams;
 struct DequantParams;
 struct MseParams;
@@ -34,6 +35,9 @@ cudaError_t launch_quantize(int fmt, int B, int K, bool mse, const QuantParams& 
 cudaError_t launch_quantize_e8m0(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 cudaError_t launch_quantize_ue4m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
 cudaError_t launch_quantize_ue5m3(int B, int K, bool mse, const QuantParams& p, int* grid_out, cudaStream_t s);
+// The batched fused quantizer (MXFP4 block 32, NVFP4 block 16); other blocks: cudaErrorInvalidValue.
+cudaError_t launch_quantize_batch_e8m0(int B, int K, const QuantBatchParams& p, cudaStream_t s);
+cudaError_t launch_quantize_batch_ue4m3(int B, int K, const QuantBatchParams& p, cudaStream_t s);
 // pdl: launch with programmatic dependent launch (never right after the memset
 // that zeroes the maximum's slot, which must complete first).
 // Quantize with MSE-optimised block scales (p.below / p.above candidate codes).

@@ -54,5 +54,29 @@ cudaError_t by_block(int B, int K, bool mse, const QuantParams& p, int* g, cudaS
     }
 }
 
+// The batched fused quantizer: grid = the resident CTAs the tiles can use, at
+// most kMaxPartialCtas (every tensor's workspace holds that many partials).
+template <int FMT, int B, int K>
+cudaError_t run_quantize_batch(const QuantBatchParams& p, cudaStream_t s)
+{
+    auto kern = quantize_batch_kernel<FMT, B, K>;
+    int64_t need = ((int64_t)p.tile0[p.count] + kWarps - 1) / kWarps;
+    if (need > kMaxPartialCtas) need = kMaxPartialCtas;
+    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
+    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
+}
+
+template <int FMT, int B>
+cudaError_t batch_by_rot(int K, const QuantBatchParams& p, cudaStream_t s)
+{
+    switch (K) {
+    case 0: return run_quantize_batch<FMT, B, 0>(p, s);
+    case 16: return run_quantize_batch<FMT, B, 16>(p, s);
+    case 32: return run_quantize_batch<FMT, B, 32>(p, s);
+    case 128: return run_quantize_batch<FMT, B, 128>(p, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace detail
 }  // namespace fp4q

@@ -226,3 +226,34 @@ def test_batched_amax_rejects_bad_arguments(fp4q):
     assert f(2, xs, rs, cs, 0, ss, 0, None) == -1                                  # non-empty tensor, no data
     xs, rs, cs, ss = arrs([A32, A32], [4, 8], [64, 128], [A32, None])
     assert f(2, xs, rs, cs, 0, ss, 1, None) == -1
+
+
+def test_batched_quantizer_rejects_bad_arguments(fp4q):
+    L = fp4q.lib()
+    f = L.fp4q_quantize_mse_dequantize_batched
+    T = fp4q.Fp4qTensor
+    ws = L.fp4q_quantize_batch_workspace_size(2)
+    assert ws >= 2 * (16 + 4096 * 32) and L.fp4q_quantize_batch_workspace_size(0) == 0
+
+    def batch(*ts):
+        return (T * len(ts))(*ts)
+
+    ok = T(A32, 4, 64, A32, A32, A32, A32, None, A32)
+    assert f(-1, batch(ok), 1, 16, 0, 3, A32, ws, None) == -2
+    assert f(0, None, 1, 16, 0, 3, None, 0, None) == 0                                  # nothing to do
+    assert f(2, None, 1, 16, 0, 3, A32, ws, None) == -1
+    assert f(2, batch(ok, ok), 1, 16, 0, 3, None, ws, None) == -1
+    assert f(2, batch(ok, ok), 1, 32, 0, 3, A32, ws, None) == -4                        # NVFP4 is block 16
+    assert f(2, batch(ok, ok), 0, 16, 0, 0, A32, ws, None) == -4                        # MXFP4 is block 32
+    assert f(2, batch(ok, ok), 2, 16, 0, 3, A32, ws, None) == -4                        # UE5M3: single calls
+    assert f(2, batch(ok, ok), 0, 32, 0, 3, A32, ws, None) == -4                        # E8M0 takes no G
+    assert f(2, batch(ok, ok), 1, 16, 12, 3, A32, ws, None) == -4                       # rot 12
+    assert f(2, batch(ok, ok), 1, 16, 0, 3, A32, ws - 8, None) == -6
+    assert f(2, batch(ok, ok), 1, 16, 0, 3, A32 + 4, ws, None) == -3
+    assert f(2, batch(ok, T(A32, 4, 60, A32, A32, A32, A32, None, A32)), 1, 16, 0, 3, A32, ws, None) == -2
+    assert f(2, batch(ok, T(A32, 4, 64, A32, A32, None, A32, None, A32)), 1, 16, 0, 3, A32, ws, None) == -1
+    assert f(2, batch(ok, T(A32, 4, 64, A32, A32, A32, None, None, A32)), 1, 16, 0, 3, A32, ws, None) == -1
+    assert f(2, batch(ok, T(A32, 4, 64, A32, A32, A32, A32, None, None)), 1, 16, 0, 3, A32, ws, None) == -1
+    assert f(2, batch(ok, T(A32 + 16, 4, 64, A32, A32, A32, A32, None, A32)), 1, 16, 0, 3, A32, ws, None) == -3
+    assert f(2, batch(ok, T(A32, 4, 64, A32 + 16, A32, A32, A32, None, A32)), 1, 16, 0, 3, A32, ws, None) == -3
+    assert f(2, batch(ok, T(A32, 4, 64, A32, A32, A32, A32, A32 + 8, A32)), 1, 16, 0, 3, A32, ws, None) == -3

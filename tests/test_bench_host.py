@@ -73,9 +73,15 @@ class _FakeLib:
 class _FakeFq:
     def __init__(self):
         self.L = _FakeLib()
+        import microscaling_fp4_quantization_block_b200 as m
+        self.Fp4qTensor = m.Fp4qTensor
 
     def lib(self):
         return self.L
+
+    @staticmethod
+    def fp4q_quantize_batch_workspace_size(count):
+        return 64 * count
 
     @staticmethod
     def fp4q_block_mse_workspace_size(rows, cols, block):
@@ -97,27 +103,35 @@ def test_weight_pass_schedule():
     pipe.step(_FakeStream())
     names = [n for n, _ in fq.L.log]
     n_nv = sum(1 for v in bench.WEIGHT_PASS_VARIANTS if v[4] == 1)
-    # one batched amax call per NVFP4 layer group, then its three quantizer calls
+    # one batched amax call per NVFP4 layer group, then one batched quantizer call on the same tensors
     assert names.count("fp4q_tensor_amax_batched") == 3 * n_nv
     assert names.count("fp4q_tensor_amax_accumulate") == 0
-    assert names.count("fp4q_quantize_mse_dequantize") == 36
-    assert pipe.launches_per_step == 36 + 3 * n_nv
+    assert names.count("fp4q_quantize_mse_dequantize_batched") == 12
+    assert names.count("fp4q_quantize_mse_dequantize") == 0
+    assert pipe.launches_per_step == 12 + 3 * n_nv
     steps = [(bench.stage_kind(st), idx) for st, _, _, idx in pipe.step_calls]
     nv_first = next(j for j, (kind, _) in enumerate(steps) if kind == "amax")
-    grp = steps[nv_first:nv_first + 4]
-    assert [k for k, _ in grp] == ["amax"] + ["quantize_mse_dequantize"] * 3
-    assert grp[0][1] == [i for _, (i,) in grp[1:]]
+    grp = steps[nv_first:nv_first + 2]
+    assert [k for k, _ in grp] == ["amax", "quantize_mse_dequantize"]
+    assert grp[0][1] == grp[1][1]
     args = pipe.step_calls[nv_first][2]
     assert args[0] == 3 and args[6] == 1                       # three tensors, accumulating into zeroed slots
     assert list(args[3]) == [items[i][1].shape[1] for i in grp[0][1]]
     assert list(args[5]) == [pipe.bufs[i]["gscale"].data_ptr() for i in grp[0][1]]
+    qargs = pipe.step_calls[nv_first + 1][2]
+    assert qargs[0] == 3 and qargs[2:6] == (1, 16, items[grp[0][1][0]][4], bench.FROM_AMAX)
+    assert [qargs[1][j].gscale for j in range(3)] == [pipe.bufs[i]["gscale"].data_ptr() for i in grp[0][1]]
+    assert [qargs[1][j].terms for j in range(3)] == [pipe.bufs[i]["terms"].data_ptr() for i in grp[0][1]]
+    mx = next(st for st in pipe.step_calls if st[0].endswith("mxfp4_rot0"))
+    assert mx[2][2:6] == (0, 32, 0, bench.NONE) and mx[2][1][0].gscale is None
     # the per-tensor form: three amax calls, then three quantizer calls on the same tensors
     fq2 = _FakeFq()
-    pipe2 = bench.Pipeline(fq2, items, "cpu", _FakeStream(), groups=groups, batch_amax=False)
+    pipe2 = bench.Pipeline(fq2, items, "cpu", _FakeStream(), groups=groups, batch_amax=False, batch_quantize=False)
     fq2.L.log.clear()
     pipe2.step(_FakeStream())
     names2 = [n for n, _ in fq2.L.log]
     assert names2.count("fp4q_tensor_amax_accumulate") == 9 * n_nv
+    assert names2.count("fp4q_quantize_mse_dequantize") == 36
     assert pipe2.launches_per_step == 36 + 9 * n_nv
     order = [(bench.stage_kind(pipe2.calls[i][k][0]), i) for i, k in pipe2.order]
     nv_first = next(j for j, (kind, _) in enumerate(order) if kind == "amax")
