@@ -847,42 +847,39 @@ struct QuantBatchParams {
 };
 
 // The last CTA to finish tensor c (a counter per tensor) sums its per-CTA
-// partials in index order (deterministic) into terms[c] = sum / n.  Every CTA
-// writes a partial for every tensor, zeros for tensors it never touched.
+// partials into terms[c] = sum / n, one warp per tensor so that the tensors'
+// sums run side by side (the same CTA is usually last for all of them).  A
+// warp sums partials lane-strided and then by a fixed shuffle tree:
+// deterministic.  Every CTA writes a partial for every tensor, zeros for
+// tensors it never touched.
 template <int NT = kThreads>
 __device__ __forceinline__ void finish_partials_batch(const QuantBatchParams& P)
 {
     constexpr int NW = NT / 32;
     __shared__ bool last[kQuantBatch];
-    __shared__ double red[NW][4];
     __threadfence();
     __syncthreads();
     if (threadIdx.x < (unsigned)P.count)
         last[threadIdx.x] = atomicInc(P.t[threadIdx.x].done, gridDim.x - 1u) == gridDim.x - 1u;
     __syncthreads();
-    for (int c = 0; c < P.count; ++c) {
-        if (!last[c]) continue;                                    // CTA-uniform
+    const int lane = threadIdx.x & 31;
+    for (int c = threadIdx.x >> 5; c < P.count; c += NW) {
+        if (!last[c]) continue;                                    // warp-uniform
         __threadfence();
         const double* partials = P.t[c].partials;
         double s[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int i = threadIdx.x; i < (int)gridDim.x; i += NT)
+        for (int i = lane; i < (int)gridDim.x; i += 32)
 #pragma unroll
             for (int k = 0; k < 4; ++k) s[k] += __ldcg(partials + (int64_t)i * 4 + k);
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], d);
-        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-        if (lane == 0)
+        if (lane == 0) {
+            const int64_t n = P.t[c].n;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) red[wid][k] = s[k];
-        __syncthreads();
-        if (threadIdx.x < 4) {
-            double t = 0.0;
-            for (int w = 0; w < NW; ++w) t += red[w][threadIdx.x];
-            P.t[c].terms[threadIdx.x] = P.t[c].n > 0 ? t / (double)P.t[c].n : 0.0;
+            for (int k = 0; k < 4; ++k) P.t[c].terms[k] = n > 0 ? s[k] / (double)n : 0.0;
         }
-        __syncthreads();
     }
 }
 

@@ -147,6 +147,9 @@ def test_weight_pass_schedule():
 def test_weight_pass_and_sweep_defaults():
     a = bench.parse_args([])
     assert a.workload == "qwen25_14b_weight_pass" and a.steps >= 3 and a.warmup >= 3
+    assert a.layers is None and not a.no_batch_quantize and not a.no_batch_amax and not a.no_graph
+    a = bench.parse_args(["--layers", "2", "--no-batch-quantize"])
+    assert a.layers == 2 and a.no_batch_quantize
     a = bench.parse_args(["--workload", "block_size_sweep_4096", "--steps", "7"])
     assert a.steps == 7 and a.warmup == bench.WORKLOAD_DEFAULTS["block_size_sweep_4096"]["warmup"]
 
