@@ -1198,11 +1198,11 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
     int64_t nbytes = 2 * p.n[0];
     int src_c = 0, cur = -1;
     float mx = 0.0f;
-    uint32_t mb = 0;                                       // max |bf16| pattern, two halves
+    uint32_t mb = 0;                                       // two halves whose magnitudes are the largest seen
     auto flush = [&]() {
         float m;
         if constexpr (K == 0) {
-            m = fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xffff0000u));
+            m = bf16x2_absmax_f32(mb);
         } else {
             // y = fp32(s c_hi + fp32(s c_lo)) rounds monotonically and symmetrically in s
             // (c_lo = 0 for K = 16), so the largest |y| is the normalised largest |s|: the
@@ -1234,12 +1234,10 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
             uint32_t w[EPT / 2];
             ring.read(s, 0, w);
             if constexpr (K == 0) {
-                // |bf16| patterns order like their values: SIMD max of both halves
+                // packed bf16 maxima of magnitudes (finite inputs: the largest magnitude's
+                // pattern; the sign bits are meaningless and masked at the flush)
 #pragma unroll
-                for (int k = 0; k < EPT / 2; ++k) {
-                    const uint32_t a = w[k] & 0x7fff7fffu;
-                    asm("max.u16x2 %0, %0, %1;" : "+r"(mb) : "r"(a));
-                }
+                for (int k = 0; k < EPT / 2; ++k) mb = bf16x2_absmax(mb, w[k]);
             } else {
                 // the raw Sylvester sums (magnitudes only: their signs do not
                 // matter); 1/sqrt(K) is applied once, to the maximum

@@ -221,17 +221,20 @@ struct TileCursor {
     }
 };
 
+// The channel maxima cmw hold, per bf16 half, a value whose magnitude is the
+// largest seen (max.xorsign.abs leaves a meaningless sign: the flush masks it).
+// Inputs are finite, so the bf16 maximum of magnitudes is the integer maximum of
+// their patterns.
 __device__ __forceinline__ void count_top(const uint32_t (&w)[4], const TopParams& p, uint32_t lo, uint32_t span,
                                           uint32_t (&cmw)[4])
 {
-    const uint32_t a[4] = {w[0] & 0x7fff7fffu, w[1] & 0x7fff7fffu, w[2] & 0x7fff7fffu, w[3] & 0x7fff7fffu};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) cmw[k] = max_u16x2(cmw[k], a[k]);
-    const uint32_t m = max_u16x2(max_u16x2(a[0], a[1]), max_u16x2(a[2], a[3]));
+    for (int k = 0; k < 4; ++k) cmw[k] = bf16x2_absmax(cmw[k], w[k]);
+    const uint32_t m = bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])) & 0x7fff7fffu;
     if (max(m & 0xffffu, m >> 16) < lo) return;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        const uint32_t v = (k & 1) ? a[k >> 1] >> 16 : a[k >> 1] & 0xffffu;
+        const uint32_t v = ((k & 1) ? w[k >> 1] >> 16 : w[k >> 1]) & 0x7fffu;
         if (v - lo < span) atomicAdd(p.hist + v, 1ull);
     }
 }
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(kThreads) outlier_top_kernel(TopParams p)
         if (cur >= 0 && p.colmax && c0 < p.cols) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint32_t c = (j & 1) ? cmw[j >> 1] >> 16 : cmw[j >> 1] & 0xffffu;
+                const uint32_t c = ((j & 1) ? cmw[j >> 1] >> 16 : cmw[j >> 1]) & 0x7fffu;
                 if (c) atomicMax(p.colmax + c0 + j, c << 16);        // |x| as fp32 bits
             }
         }
