@@ -35,9 +35,9 @@ cudaError_t run_mse(const MseParams& p, int* grid_out, cudaStream_t s)
     auto kern = block_mse_kernel<B, K>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (need > partial_slots(p.n)) need = partial_slots(p.n);
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
+    const int grid = grid_for((const void*)kern, ring_smem_bytes<K>(), need);
     *grid_out = grid;
-    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
+    return launch_pdl(kern, grid, kThreads, ring_smem_bytes<K>(), s, p);
 }
 
 #define FP4Q_BK_SWITCH(B, K, CALL)                                                   \

@@ -336,6 +336,16 @@ __device__ __forceinline__ void upk(f32x2 v, float& a, float& b)
 {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
 }
+
+// 16 bytes of shared memory as two fp32 pairs, and back.
+__device__ __forceinline__ void sts_pairs(uint32_t smem_addr, f32x2 a, f32x2 b)
+{
+    asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(smem_addr), "l"(a), "l"(b) : "memory");
+}
+__device__ __forceinline__ void lds_pairs(uint32_t smem_addr, f32x2& a, f32x2& b)
+{
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(smem_addr) : "memory");
+}
 __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
 {
     f32x2 r;
@@ -442,8 +452,10 @@ __device__ __forceinline__ ScaleConsts scale_consts(float G)
 // Sylvester Hadamard transform of every run of CH consecutive values (natural
 // order: y_i = sum_j (-1)^popcount(i & j) x_j): the distance-1 stage mixes the
 // two halves of each pair, the others combine whole pairs.  FIRST = false
-// skips the distance-1 stage (done already by unpack_fwht2).
-template <int N, int CH, bool FIRST = true>
+// skips the distance-1 stage (done already by unpack_fwht2); the pair stages
+// run at distances H0, 2 H0, ... below CH (H0 > 2: the stages of the lower
+// index bits are done already).
+template <int N, int CH, bool FIRST = true, int H0 = 2>
 __device__ __forceinline__ void fwht_inreg(f32x2 (&p)[N / 2])
 {
     if constexpr (FIRST && CH >= 2) {
@@ -455,7 +467,7 @@ __device__ __forceinline__ void fwht_inreg(f32x2 (&p)[N / 2])
         }
     }
 #pragma unroll
-    for (int h = 2; h < CH; h <<= 1) {
+    for (int h = H0; h < CH; h <<= 1) {
 #pragma unroll
         for (int i = 0; i < N; i += 2) {
             if ((i & h) == 0) {
@@ -489,27 +501,6 @@ __device__ __forceinline__ void unpack_fwht2(const uint32_t (&w)[N / 2], f32x2 (
             : "=f"(s), "=f"(d)
             : "r"(w[k]), "f"(lo));
         p[k] = pk(s, d);
-    }
-}
-
-// Butterfly stages across LANES consecutive lanes (each lane holding the next
-// N values of the run): lane bit d pairs lane l with l ^ d; the lower lane
-// keeps a + b, the upper one a - b, a being the lower lane's value; both are
-// other + sign * own with sign = +1 / -1.
-template <int N, int LANES>
-__device__ __forceinline__ void fwht_xlane(f32x2 (&p)[N / 2], int lane)
-{
-#pragma unroll
-    for (int d = 1; d < LANES; d <<= 1) {
-        const float sg = (lane & d) ? -1.0f : 1.0f;
-        const f32x2 sg2 = pk(sg, sg);
-#pragma unroll
-        for (int k = 0; k < N / 2; ++k) {
-            float a, b;
-            upk(p[k], a, b);
-            const f32x2 other = pk(__shfl_xor_sync(0xffffffffu, a, d), __shfl_xor_sync(0xffffffffu, b, d));
-            p[k] = fma2(p[k], sg2, other);            // exact: sign * own is exact
-        }
     }
 }
 

@@ -39,12 +39,16 @@ struct GscaleParams {
     double* errors;             // out (optional): per-candidate per-tensor MSE, index j + below
 };
 
-// Dynamic shared memory after the ring: per-candidate scale tables, constants
-// and the per-warp error accumulators.
+// Dynamic shared memory after the ring (and the rotation scratch): per-candidate
+// scale tables, constants and the per-warp error accumulators.
 constexpr int kTabBytes = kMaxCand * 256 * (int)sizeof(float2);
 constexpr int kConstBytes = kMaxCand * (int)sizeof(float4);
 constexpr int kAccBytes = kWarps * kMaxCand * (int)sizeof(double);
-constexpr int kSmemBytes = kRingBytesPerCta + kTabBytes + kConstBytes + kAccBytes;
+template <int K>
+constexpr int smem_bytes()
+{
+    return ring_smem_bytes<K>() + kTabBytes + kConstBytes + kAccBytes;
+}
 
 // Squared error of one unit under one candidate scale: the unit's share of its
 // blocks' errors (fp32 sums of fp32 terms, as the fused MSE forms them).
@@ -99,9 +103,10 @@ __global__ void __launch_bounds__(kThreads, 1) gscale_search_kernel(GscaleParams
     pdl_wait();
     pdl_release();
     extern __shared__ __align__(128) uint8_t smem[];
-    float2* tabs = reinterpret_cast<float2*>(smem + kRingBytesPerCta);
-    float4* consts = reinterpret_cast<float4*>(smem + kRingBytesPerCta + kTabBytes);
-    double* wacc = reinterpret_cast<double*>(smem + kRingBytesPerCta + kTabBytes + kConstBytes);
+    constexpr int kTab0 = ring_smem_bytes<K>();
+    float2* tabs = reinterpret_cast<float2*>(smem + kTab0);
+    float4* consts = reinterpret_cast<float4*>(smem + kTab0 + kTabBytes);
+    double* wacc = reinterpret_cast<double*>(smem + kTab0 + kTabBytes + kConstBytes);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int nc = p.below + p.above + 1;
     const float amax = *p.amax;
@@ -121,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) gscale_search_kernel(GscaleParams
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const XRing ring = warp_ring<XRing>(smem);
+    const XRing ring = warp_ring<XRing, K>(smem);
     const float nz = __uint_as_float(0x80000000u | (uint32_t)((uint64_t)p.n >> 63));
     using S = UnitShape<B, K>;
     stream_tiles(ring, reinterpret_cast<const uint8_t*>(p.x), 2 * p.n, n_tiles, warp, n_warps, lane,
@@ -192,8 +197,8 @@ cudaError_t run_gscale(const GscaleParams& p, cudaStream_t s)
     auto kern = gscale_search_kernel<FMT, B, K>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (need > kMaxPartialCtas) need = kMaxPartialCtas;
-    const int grid = grid_for((const void*)kern, kSmemBytes, need);
-    kern<<<grid, kThreads, kSmemBytes, s>>>(p);
+    const int grid = grid_for((const void*)kern, smem_bytes<K>(), need);
+    kern<<<grid, kThreads, smem_bytes<K>(), s>>>(p);
     return cudaGetLastError();
 }
 

@@ -7,10 +7,11 @@
 // Work decomposition.  A lane owns "units" of 32 consecutive elements; the 32
 // lanes of a warp own the 32 consecutive units of a 1024-element "tile"
 // (quantize, amax, MSE), so blocks of 8, 16 or 32 sit inside one lane, wider
-// blocks and rotation runs span adjacent lanes (maxima combined with
-// shuffles, butterflies finished across lanes).  Warps walk tiles in a
-// grid-stride loop with the same trip count for every lane (lanes past the
-// end hold zeros), so shuffles always see the whole warp.
+// blocks span adjacent lanes (maxima combined with shuffles), and a 128-wide
+// rotation run spans 4 lanes, which trade halves of it through shared memory
+// (unit_sums).  Warps walk tiles in a grid-stride loop with the same trip
+// count for every lane (lanes past the end hold zeros), so shuffles and warp
+// barriers always see the whole warp.
 //
 // Memory pipeline.  The streamed input goes through a per-warp ring of
 // NSTAGE tiles in shared memory filled with 16-byte cp.async copies: while a
@@ -69,16 +70,31 @@ struct Ring {
     uint32_t wr[CPL];              // shared offset (in a sub-tile) of the chunk this lane copies, per c
     uint32_t rd[CPL];              // shared offset (in a sub-tile) of this lane's c-th chunk
 
-    // smem chunk of global chunk j of a sub-tile: XOR swizzle that keeps both
-    // the contiguous copies and the per-lane 128-bit reads conflict free.
-    static __device__ __forceinline__ int swz(int j) { return CPL == 1 ? j : (j ^ ((j >> 3) & (CPL - 1))); }
+    // smem chunk of global chunk j of a sub-tile: an XOR swizzle, constant over
+    // each aligned group of 8 chunks, that keeps conflict free (8 lanes of a
+    // 128-bit access cover the 8 distinct 16-byte bank groups) the contiguous
+    // copies, the per-lane reads of a unit and, with 4 chunks per lane, the
+    // reads of the 128-element run layout below: group m = (j / 8) mod 4 is
+    // XORed with m ^ ((m & 2) << 1), i.e. 0, 1, 6, 7.
+    static __device__ __forceinline__ int swz(int j)
+    {
+        if constexpr (CPL == 1) return j;
+        if constexpr (CPL == 2) return j ^ ((j >> 3) & 1);
+        const int m = (j >> 3) & 3;
+        return j ^ (m ^ ((m & 2) << 1));
+    }
 
-    __device__ __forceinline__ Ring(uint32_t b, int lane) : base(b)
+    // runs128 (4 chunks per lane only): the lanes 4g .. 4g+3 that own the
+    // 128-element run g of a tile read it interleaved, lane 4g + c getting the
+    // chunks (8 elements each) 4j + c of the run, j = 0..3, in place of its own
+    // unit's four; see unit_sums.
+    __device__ __forceinline__ Ring(uint32_t b, int lane, bool runs128 = false) : base(b)
     {
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             wr[c] = 16u * (uint32_t)swz(lane + 32 * c);
-            rd[c] = 16u * (uint32_t)swz(CPL * lane + c);
+            const int j = (CPL == 4 && runs128) ? 16 * (lane >> 2) + 4 * c + (lane & 3) : CPL * lane + c;
+            rd[c] = 16u * (uint32_t)swz(j);
         }
     }
 
@@ -131,11 +147,40 @@ struct Ring {
     }
 };
 
-template <typename R>
+// This warp's ring; K: the rotation of the kernel's units (a rotation wider
+// than a unit reads its runs interleaved, see unit_sums).
+template <typename R, int K = 0>
 __device__ __forceinline__ R warp_ring(uint8_t* smem)
 {
     return R((uint32_t)__cvta_generic_to_shared(smem) + (uint32_t)((threadIdx.x >> 5) * kRingBytesPerWarp),
-             threadIdx.x & 31);
+             threadIdx.x & 31, K > EPT);
+}
+
+// Shared-memory scratch of a rotation wider than a unit (the lane transpose
+// in unit_sums): 131 16-byte chunks per warp, in the dynamic shared memory
+// right after the ring.  A kernel that instantiates such a rotation launches
+// with ring_smem_bytes<K>() of dynamic shared memory (or more, other regions
+// following the scratch).
+constexpr int kRotScratchBytesPerWarp = 131 * 16;
+
+template <int K>
+__host__ __device__ constexpr int rot_scratch_bytes()
+{
+    return K > EPT ? kRotScratchBytesPerWarp * kWarps : 0;
+}
+
+template <int K>
+__host__ __device__ constexpr int ring_smem_bytes()
+{
+    return kRingBytesPerCta + rot_scratch_bytes<K>();
+}
+
+extern __shared__ __align__(128) uint8_t smem_dynamic[];
+
+__device__ __forceinline__ uint32_t rot_scratch()
+{
+    return (uint32_t)__cvta_generic_to_shared(smem_dynamic) + (uint32_t)kRingBytesPerCta +
+           (uint32_t)((threadIdx.x >> 5) * kRotScratchBytesPerWarp);
 }
 
 // Ring pipeline driver: calls body(tile, stage) for every tile of this warp,
@@ -204,17 +249,50 @@ __device__ __forceinline__ void unpack_unit(const uint32_t (&w)[EPT / 2], f32x2 
     for (int k = 0; k < EPT / 2; ++k) p[k] = pk(bf16_lo(w[k]), bf16_hi_fp(w[k]));
 }
 
-// The Sylvester sums of a unit's runs of K elements (K > 0): the part of a run
-// inside the unit in registers, the rest across lanes.  The odd positions come
-// out negated (see unpack_fwht2); only magnitudes are read from the result, or
-// normalise_signed restores the signs.
+// Lane transpose of the 128-element runs, half a unit at a time.  Lane
+// L = 4g + c holds in p[4j + i] the pairs of elements 32j + 8c + 2i, +1 of run
+// g (row j of the run as 4 rows of 32, its 8-element column c); afterwards
+// lane 4g + j holds in p[4c + i] those of row j, columns c = 0..3: its own
+// 32 consecutive elements.  Round h moves pairs i = 2h, 2h + 1 through
+// scratch chunk R + 33 c for (row R = 4g + j of the warp, column c): every
+// 16-byte store (fixed j) and load (fixed c) of 8 lanes hits 8 distinct bank
+// groups, and each round refills exactly the registers it sent.  (Both halves
+// at once, through two scratch regions and one barrier, measured slower.)
+__device__ __forceinline__ void transpose_runs128(f32x2 (&p)[EPT / 2], int lane, uint32_t scr)
+{
+    const uint32_t rd = scr + 16u * (uint32_t)lane;              // row L, column c at + 528 c
+    const uint32_t wr = rd + 512u * (uint32_t)(lane & 3);        // row 4g + j at + 16 j, column c
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        __syncwarp();                                            // the scratch's last readers are done
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sts_pairs(wr + 16u * j, p[4 * j + 2 * h], p[4 * j + 2 * h + 1]);
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) lds_pairs(rd + 528u * c, p[4 * c + 2 * h], p[4 * c + 2 * h + 1]);
+    }
+}
+
+// The Sylvester sums of a unit's runs of K elements (K > 0).  The odd
+// positions come out negated (see unpack_fwht2); only magnitudes are read
+// from the result, or normalise_signed restores the signs.
+// K <= 32: the runs lie inside the unit, all in registers.
+// K = 128: a run spans 4 lanes.  The ring hands each lane the run's
+// interleaved chunks (Ring, runs128), so that the stages of element bits 0-2
+// and 5-6 run in registers; a transpose through shared memory (the warp's
+// rot_scratch) gives each lane its own 32 elements back, and the stages of
+// bits 3-4 run in registers too.  Same sums as the stages in bit order, with
+// the roundings of a different order.
 template <int K>
 __device__ __forceinline__ void unit_sums(const uint32_t (&w)[EPT / 2], f32x2 (&p)[EPT / 2], int lane)
 {
-    static_assert(K >= 2, "rotation runs of at least two elements");
+    static_assert(K >= 2 && (K <= EPT || K == 4 * EPT), "rotation runs of 2..32 or 128 elements");
     unpack_fwht2<EPT>(w, p);
     fwht_inreg<EPT, (K < EPT ? K : EPT), false>(p);
-    if constexpr (K > EPT) fwht_xlane<EPT, K / EPT>(p, lane);
+    if constexpr (K > EPT) {
+        transpose_runs128(p, lane, rot_scratch());
+        fwht_inreg<EPT, EPT, false, 8>(p);
+    }
 }
 
 // y = s / sqrt(K) rounded to fp32, the odd positions' signs restored by
@@ -787,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, (MSE || FMT != kE8M0) ? 2 : 3) quant
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const XRing ring = warp_ring<XRing>(smem_ring);
+    const XRing ring = warp_ring<XRing, K>(smem_ring);
 
     // Evict-first in L2 for what the step does not read again, so that it does
     // not push out lines that are: x where this is its last read (MSE fused), and
@@ -897,7 +975,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_batch_kernel(const __gri
     const int32_t n_tiles = P.tile0[P.count];
     const int32_t warp = (int32_t)(blockIdx.x * (kThreads / 32)) + warp_in;
     const int32_t n_warps = (int32_t)(gridDim.x * (kThreads / 32));
-    const XRing ring = warp_ring<XRing>(smem_ring);
+    const XRing ring = warp_ring<XRing, K>(smem_ring);
     const uint64_t pol = l2_evict_first();
 
     // ---- the tiles of all tensors; a warp's tiles rise, so its tensors do too:
@@ -1126,7 +1204,7 @@ __global__ void __launch_bounds__(kThreads, 2) search_kernel(QuantParams p)
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const XRing ring = warp_ring<XRing>(smem_ring);
+    const XRing ring = warp_ring<XRing, K>(smem_ring);
 
     float G = 1.0f;
     if (FMT != kE8M0 && p.gsrc != nullptr) {
@@ -1177,7 +1255,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxParams p)
     const int64_t n_tiles = p.tile0[p.count];
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const XRing ring = warp_ring<XRing>(smem_ring);
+    const XRing ring = warp_ring<XRing, K>(smem_ring);
     // A warp's tiles rise, so its tensors do too: one cursor for the copies issued
     // ahead and one for the tile being reduced, each holding its tensor's tile range
     // (and source) in registers so that a tile of the same tensor costs one compare.
@@ -1662,7 +1740,7 @@ __global__ void __launch_bounds__(kThreads) block_mse_kernel(MseParams p)
     const int64_t n_tiles = (p.n + 32 * EPT - 1) / (32 * EPT);
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const XRing ring = warp_ring<XRing>(smem_ring);
+    const XRing ring = warp_ring<XRing, K>(smem_ring);
     const float G = (p.fmt != kE8M0 && p.gsrc != nullptr) ? *p.gsrc : 1.0f;
 
     double acc_total = 0.0, acc_nonmax = 0.0, acc_max = 0.0, acc_zero = 0.0;

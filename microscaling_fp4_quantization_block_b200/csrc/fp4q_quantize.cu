@@ -104,9 +104,9 @@ cudaError_t run_amax(const AmaxParams& p, cudaStream_t s, bool pdl)
 {
     auto kern = amax_kernel<K>;
     const int64_t tiles = p.tile0[p.count];
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, (tiles + kWarps - 1) / kWarps);
-    if (pdl) return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
-    kern<<<grid, kThreads, kRingBytesPerCta, s>>>(p);
+    const int grid = grid_for((const void*)kern, ring_smem_bytes<K>(), (tiles + kWarps - 1) / kWarps);
+    if (pdl) return launch_pdl(kern, grid, kThreads, ring_smem_bytes<K>(), s, p);
+    kern<<<grid, kThreads, ring_smem_bytes<K>(), s>>>(p);
     return cudaGetLastError();
 }
 

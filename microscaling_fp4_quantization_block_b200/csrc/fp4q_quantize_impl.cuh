@@ -16,9 +16,9 @@ cudaError_t run_quantize(const QuantParams& p, int* grid_out, cudaStream_t s)
     auto kern = quantize_kernel<FMT, B, K, MSE, DQ>;
     int64_t need = ring_ctas_needed(p.n, EPT);
     if (MSE && need > partial_slots(p.n)) need = partial_slots(p.n);
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
+    const int grid = grid_for((const void*)kern, ring_smem_bytes<K>(), need);
     if (grid_out) *grid_out = grid;
-    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
+    return launch_pdl(kern, grid, kThreads, ring_smem_bytes<K>(), s, p);
 }
 
 template <int FMT, int B, int K>
@@ -62,8 +62,8 @@ cudaError_t run_quantize_batch(const QuantBatchParams& p, cudaStream_t s)
     auto kern = quantize_batch_kernel<FMT, B, K>;
     int64_t need = ((int64_t)p.tile0[p.count] + kWarps - 1) / kWarps;
     if (need > kMaxPartialCtas) need = kMaxPartialCtas;
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, need);
-    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
+    const int grid = grid_for((const void*)kern, ring_smem_bytes<K>(), need);
+    return launch_pdl(kern, grid, kThreads, ring_smem_bytes<K>(), s, p);
 }
 
 template <int FMT, int B>

@@ -11,8 +11,8 @@ template <int FMT, int B, int K>
 cudaError_t run_search(const QuantParams& p, cudaStream_t s)
 {
     auto kern = search_kernel<FMT, B, K>;
-    const int grid = grid_for((const void*)kern, kRingBytesPerCta, ring_ctas_needed(p.n, EPT));
-    return launch_pdl(kern, grid, kThreads, kRingBytesPerCta, s, p);
+    const int grid = grid_for((const void*)kern, ring_smem_bytes<K>(), ring_ctas_needed(p.n, EPT));
+    return launch_pdl(kern, grid, kThreads, ring_smem_bytes<K>(), s, p);
 }
 
 template <int FMT, int B>

@@ -41,16 +41,36 @@ def _check(fq, x, fmt, block, rot, below, above):
     _, _, og, oerrs = oracle.global_scale_search(xb, fmt, block, rot, below, above)
     tol = (block + 4) * 2.0 ** -24 if rot == 0 else 1e-5
     assert np.allclose(errs, oerrs, rtol=tol, atol=0.0), np.max(np.abs(errs - oerrs) / oerrs)
+    # the candidate grids: the oracle's from its G0, the kernel's from its own
+    # (equal unrotated; rotated, its maximum comes from fp32 butterflies, so its
+    # G0 may differ from the oracle's through that maximum, as the rotated-path
+    # rule allows: a few fp32 ulps)
+    g0, g0k = _g0(xb, rot), _g0_kernel(fq, x, rot)
+    if rot == 0:
+        assert np.float32(g0k) == np.float32(g0), (g0k, g0)
+    else:
+        assert abs(g0k - g0) <= 2.0 ** -21 * g0, (g0k, g0)
     if np.float32(g) != np.float32(og):
         # only between candidates whose exact errors agree to the kernel's rounding
-        jg = [j for j in range(-below, above + 1)
-              if np.float32(g) == np.float32(np.float64(_g0(xb, rot)) * (16 + j) / 16)]
-        jo = [j for j in range(-below, above + 1)
-              if np.float32(og) == np.float32(np.float64(_g0(xb, rot)) * (16 + j) / 16)]
+        jg = [j for j in range(-below, above + 1) if np.float32(g) == _candidate(g0k, j)]
+        jo = [j for j in range(-below, above + 1) if np.float32(og) == _candidate(g0, j)]
         assert jg and jo, (g, og)
-        e1, e2 = oerrs[jg[0] + below], oerrs[jo[0] + below]
-        assert abs(e1 - e2) <= 2 * tol * max(e1, e2), (g, og, e1, e2)
+        if jg[0] != jo[0]:
+            e1, e2 = oerrs[jg[0] + below], oerrs[jo[0] + below]
+            assert abs(e1 - e2) <= 2 * tol * max(e1, e2), (g, og, e1, e2)
     return g, og, errs
+
+
+def _candidate(g0, j):
+    """Candidate j of the per-tensor scale grid: fp32(G0 (16 + j) / 16)."""
+    return np.float32(np.float32(g0) * np.float32((16 + j) / 16))
+
+
+def _g0_kernel(fq, x, rot):
+    """The kernel's max-rule G0: its tensor maximum (of the rotated values, for
+    rot > 0) / 2688, correctly rounded in fp32, 1 for an all-zero tensor."""
+    amax = float(fq.fp4q_tensor_amax(x.cuda(), rot).item())
+    return float(np.float32(amax) / np.float32(2688.0)) if amax > 0 else 1.0
 
 
 def _g0(xb, rot):
