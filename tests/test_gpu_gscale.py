@@ -6,8 +6,11 @@ the kernel on sums of fp32 block errors (each within (b + 4) 2^-24 relative of
 the exact block error).  So:
 - every per-candidate error within (b + 4) 2^-24 relative of the oracle's
   (unrotated), 1e-5 (rotated: fp32 butterflies against an fp64 rotation);
-- the chosen G equal to the oracle's, unless the oracle's exact errors of the
-  two choices agree within twice that bound (then either is right);
+- the kernel's own max-rule G0 equal to the oracle's (unrotated), or within
+  2^-21 relative (rotated: its tensor maximum comes from fp32 butterflies);
+- the chosen candidate index equal to the oracle's, each on its own G0 grid,
+  unless the oracle's exact errors of the two choices agree within twice that
+  bound (then either is right);
 - the hand-worked two-block tensors of the oracle's pins give their hand
   results on the GPU too.
 """
