@@ -162,3 +162,24 @@ def test_reference_arm_sweep(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["config"]["workload"] == "block_size_sweep_4096"
+
+
+def test_ncu_traffic_follows_the_kernel_sources(monkeypatch):
+    """The roofline's measured traffic is read from the committed counters only
+    while the kernel sources they were taken on are unchanged; otherwise, and
+    for a kernel without counters, the line carries null."""
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
+        table = json.load(f)
+    wl = "qwen25_14b_weight_pass"
+    for kernel, e in table[wl].items():
+        assert e["csrc_files"] and 1.9 < e["dram_bytes_per_element"] < 5.0, kernel
+        v = bench.ncu_traffic(kernel, wl)
+        if e["csrc_sha"] == bench.csrc_hash(e["csrc_files"]):
+            assert v == e["dram_bytes_per_element"], kernel
+        else:
+            assert v is None, kernel
+    assert bench.ncu_traffic("no_such_kernel@x", wl) is None
+    assert bench.ncu_traffic("amax@nvfp4_rot0", "no_such_workload") is None
+    monkeypatch.setattr(bench, "csrc_hash", lambda files=None: "0" * 16)
+    assert all(bench.ncu_traffic(k, wl) is None for k in table[wl])
